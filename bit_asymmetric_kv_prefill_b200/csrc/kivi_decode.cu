@@ -1,0 +1,711 @@
+// kivi_decode.cu -- split-K flash-decoding attention over the packed 2-bit
+// KIVI cache plus its full-precision residual.
+//
+// One decode query per head attends to every cached token: the grouped 2-bit
+// history and the newest r <= R residual tokens (KIVI: A Tuning-Free Asymmetric
+// 2bit Quantization for KV Cache, Key points; record
+// kv-efficiency/kivi-2bit-llama2-13b-mha-4k, "KV bytes basis").  The pass is a
+// memory-bound GEMV, so it runs on the CUDA cores:
+//
+//  * Work split: the flattened (sequence, item) list, items being 32-token
+//    groups and 6-token residual slices, is cut into equal contiguous weight
+//    ranges, one per warp of a one-CTA-per-SM grid (Split in kivi_common.cuh).
+//  * Each warp streams its items through a private ring of shared-memory
+//    stages filled by cp.async.bulk (the bulk-copy engine) and completed on
+//    mbarriers; every wait is bounded and reports through the status word.
+//  * Keys: per group the lane folds the per-channel scale into the query,
+//    q'_d = q_d * s_d, and the zero into one bias b = sum_d q_d z_d, so that
+//    q.k = sum_d q'_d c_d + b.  Codes are turned into floats by OR-ing the
+//    2-bit field into a float's mantissa under a fixed exponent and
+//    subtracting the exponent's power of two (exact), two at a time with
+//    packed fp32x2 adds and FMAs.
+//  * Values: p'_{t,j} = p_t s_{t,j} and sum_t p_t z_{t,j} likewise fold the
+//    per-token scale and zero; lanes own channels.
+//  * Softmax is online in fp32 in the log2 domain (the query carries
+//    log2(e)/sqrt(D)); the running max is only raised when a score exceeds it
+//    by more than 8, which keeps all rescaling rare.
+//  * Each warp writes one unnormalised partial (o, m, l) per sequence it
+//    touches; the warp that arrives last on the sequence's ticket (atomic
+//    counter, no waiting) merges them with a log-sum-exp combine and writes
+//    the fp32 output.
+//  * Pre-RoPE caches dequantize keys explicitly and rotate them at their
+//    absolute positions (KIVI article, paragraph 4; KVQuant summary,
+//    "Pre-RoPE Key Quantization").
+#include <cuda_runtime.h>
+
+#include "kivi_common.cuh"
+#include "kivi_internal.h"
+
+namespace kivi {
+
+constexpr unsigned FULL = 0xffffffffu;
+constexpr int kStages = 3;
+constexpr float kRescaleSlack = 8.0f;
+constexpr long long kWaitLimit = 1LL << 22;
+
+// ---- PTX wrappers ----------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, int count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                         uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// ---- code extraction ---------------------------------------------------------
+// Slot i of a word sits at bits [2i, 2i+1].  Slots 0..10 are read in place,
+// slots 11..15 from the word shifted right by 22.  With the field at bit p of
+// the mantissa and biased exponent 150 - p, the float equals 2^(23-p) + c.
+__device__ __forceinline__ float code_raw(uint32_t w, uint32_t w22, int i)
+{
+    const int p = i <= 10 ? 2 * i : 2 * i - 22;
+    const uint32_t src = i <= 10 ? w : w22;
+    return __uint_as_float((src & (3u << p)) | ((uint32_t)(150 - p) << 23));
+}
+__device__ __forceinline__ float code_magic(int i)
+{
+    const int p = i <= 10 ? 2 * i : 2 * i - 22;
+    return -__uint_as_float((uint32_t)(150 - p) << 23);
+}
+// Exact (c_i, c_{i+1}) as floats.
+__device__ __forceinline__ float2 code_pair(uint32_t w, uint32_t w22, int i)
+{
+    return fadd2(make_float2(code_raw(w, w22, i), code_raw(w, w22, i + 1)),
+                 make_float2(code_magic(i), code_magic(i + 1)));
+}
+
+template <int DT>
+__device__ __forceinline__ float to_f(uint16_t b)
+{
+    if constexpr (DT == 1) return __uint_as_float((uint32_t)b << 16);
+    else return __half2float(__ushort_as_half(b));
+}
+__device__ __forceinline__ float f16f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
+    return x;
+}
+__device__ __forceinline__ float warp_max(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, o));
+    return x;
+}
+
+// ---- shared-memory plan per warp ------------------------------------------------
+template <int D, int HG, bool ROPE>
+struct WarpSmem {
+    using L = Layout<D>;
+    static constexpr int QPS = D / 4 + 4;           // padded q' slice (floats)
+    static constexpr int PPS = 36;                  // padded p' row (floats)
+    static constexpr int RING = 0;                  // kStages x GB
+    static constexpr int QP = kStages * L::GB;      // float [HG][4][QPS]
+    static constexpr int PP = QP + HG * 4 * QPS * 4;          // float [HG][NJ][PPS]
+    static constexpr int QS = PP + HG * L::NJ * PPS * 4;      // float [HG][D]
+    static constexpr int SZ = QS + HG * D * 4;                // float2 [4][D/4] (RoPE)
+    static constexpr int BAR = SZ + (ROPE ? D * 8 : 0);       // uint64 [kStages]
+    static constexpr int BYTES = (BAR + kStages * 8 + 15) / 16 * 16;
+};
+
+template <int D, int HG, bool ROPE>
+struct DecodeShape {
+    static constexpr int PER_WARP = WarpSmem<D, HG, ROPE>::BYTES;
+    static constexpr int MAXW = 232448 / PER_WARP;
+    static constexpr int NW = MAXW > 16 ? 16 : MAXW;
+    static constexpr int SMEM = NW * PER_WARP;
+};
+
+// ---- the kernel ---------------------------------------------------------------
+template <int D, int HG, int DT, bool ROPE>
+__global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
+    decode_kernel(const DecodeParams p)
+{
+    using L = Layout<D>;
+    using W = WarpSmem<D, HG, ROPE>;
+    constexpr int NW = DecodeShape<D, HG, ROPE>::NW;
+    constexpr int CPL = L::CPL, NJ = L::NJ, KW = L::KW, HALF = L::HALF;
+    constexpr int PSTRIDE = D + 4;
+
+    extern __shared__ __align__(128) unsigned char smem_all[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long gw = (long long)blockIdx.x * NW + warp;
+    if (gw >= p.warps) return;  // warp-uniform
+
+    unsigned char *ws = smem_all + warp * W::BYTES;
+    unsigned char *ring = ws + W::RING;
+    float *qp = (float *)(ws + W::QP);
+    float *pp = (float *)(ws + W::PP);
+    float *qs = (float *)(ws + W::QS);
+    float2 *sz = (float2 *)(ws + W::SZ);
+    const uint32_t bar0 = smem_addr(ws + W::BAR);
+
+    Split sp;
+    sp.init(p.seqs, p.n_groups, p.r, p.wg, p.wr, p.warps);
+    const long long lo = sp.lo(gw), hi = sp.lo(gw + 1);
+    const long long s_first = lo / sp.C, s_last = (hi - 1) / sp.C;
+
+    if (lane == 0) {
+        for (int i = 0; i < kStages; ++i) mbar_init(bar0 + 8 * i, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+
+    // Prefetch iterator over the warp's items, possibly across sequences.
+    long long pf_s = s_first, pf_i = 0, pf_e = 0;
+    sp.items(pf_s, gw, &pf_i, &pf_e);
+    auto pf_advance = [&]() {
+        while (pf_i >= pf_e && pf_s < s_last) {
+            ++pf_s;
+            sp.items(pf_s, gw, &pf_i, &pf_e);
+        }
+    };
+    pf_advance();
+    long long issued = 0, consumed = 0;
+    auto issue_next = [&]() {
+        pf_advance();
+        if (pf_i >= pf_e) return;
+        const int st = (int)(issued % kStages);
+        if (lane == 0) {
+            const uint32_t bar = bar0 + 8 * st;
+            const uint32_t dst = smem_addr(ring + st * L::GB);
+            if (pf_i < p.n_groups) {
+                const uint8_t *src = p.packed + (pf_s * p.ngcap + pf_i) * (long long)L::GB;
+                mbar_expect_tx(bar, L::GB);
+                bulk_g2s(dst, src, L::GB, bar);
+            } else {
+                const int t0 = (int)(pf_i - p.n_groups) * kResTok;
+                const int nt = min(kResTok, p.r - t0);
+                const uint32_t bytes = (uint32_t)nt * D * 2;
+                const long long row = pf_s * (long long)p.R + t0;
+                mbar_expect_tx(bar, 2 * bytes);
+                bulk_g2s(dst, p.resK + row * D, bytes, bar);
+                bulk_g2s(dst + kResTok * D * 2, p.resV + row * D, bytes, bar);
+            }
+        }
+        ++issued;
+        ++pf_i;
+    };
+    for (int i = 0; i < kStages; ++i) issue_next();
+
+    bool failed = false;
+    auto wait_stage = [&](long long k) -> bool {
+        const uint32_t bar = bar0 + 8 * (int)(k % kStages);
+        const uint32_t par = (uint32_t)((k / kStages) & 1);
+        for (long long it = 0; it < kWaitLimit; ++it)
+            if (__all_sync(FULL, mbar_try_wait(bar, par))) return true;
+        return false;
+    };
+
+    const int tq = lane >> 2, cs = lane & 3;   // K mapping: 4 tokens x slice cs
+    const int pcs = lane >> 3;                  // q' writer: permuted slice
+    const int pL0 = (lane & 7) * CPL;           //   and first local index
+    const int jl = lane * CPL / 32;             // V mapping: value group of lane
+
+    for (long long s = s_first; s <= s_last && !failed; ++s) {
+        long long i0, i1;
+        sp.items(s, gw, &i0, &i1);
+        const long long b = s / p.H_kv;
+        const int hk = (int)(s % p.H_kv);
+        const uint16_t *qg = p.q + (b * p.H_q + (long long)hk * HG) * D;
+
+        // Scaled query in shared memory (fp32) and the lane's q' inputs.
+        __syncwarp();
+        for (int i = lane; i < HG * D; i += 32) qs[i] = to_f<DT>(qg[i]) * p.qscale;
+        __syncwarp();
+        float qreg[HG][CPL];
+#pragma unroll
+        for (int h = 0; h < HG; ++h)
+#pragma unroll
+            for (int e = 0; e < CPL; ++e) qreg[h][e] = qs[h * D + k_channel<D>(pcs, pL0 + e)];
+
+        float m[HG], lsum[HG], zacc[HG][NJ];
+        float2 accV[HG][CPL / 2];
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+            m[h] = -INFINITY;
+            lsum[h] = 0.f;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) zacc[h][j] = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPL / 2; ++c) accV[h][c] = make_float2(0.f, 0.f);
+        }
+
+        // Online softmax update with the lane's score s_h for one token (or
+        // -inf), valid for the lane when `own` holds.
+        auto softmax_step = [&](float (&sc)[HG], float (&pr)[HG], bool own) {
+#pragma unroll
+            for (int h = 0; h < HG; ++h) {
+                const bool need = sc[h] > m[h] + kRescaleSlack;
+                if (__any_sync(FULL, need)) {
+                    const float mn = fmaxf(m[h], warp_max(sc[h]));
+                    const float alpha = ex2(m[h] - mn);
+                    lsum[h] *= alpha;
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j) zacc[h][j] *= alpha;
+#pragma unroll
+                    for (int c = 0; c < CPL / 2; ++c) {
+                        accV[h][c].x *= alpha;
+                        accV[h][c].y *= alpha;
+                    }
+                    m[h] = mn;
+                }
+                pr[h] = ex2(sc[h] - m[h]);
+                if (own) lsum[h] += pr[h];
+            }
+        };
+
+        for (long long it = i0; it < i1; ++it) {
+            if (!wait_stage(consumed)) {
+                failed = true;
+                break;
+            }
+            const unsigned char *st = ring + (int)(consumed % kStages) * L::GB;
+            if (it < p.n_groups) {
+                // ---------------- quantized group of 32 tokens ----------------
+                const uint16_t *km = (const uint16_t *)(st + L::KM + lane * (D / 8));
+                float bias[HG];
+                if constexpr (!ROPE) {
+#pragma unroll
+                    for (int h = 0; h < HG; ++h) {
+                        float bp = 0.f;
+                        float qv[CPL];
+#pragma unroll
+                        for (int e = 0; e < CPL; ++e) {
+                            qv[e] = qreg[h][e] * f16f(km[e]);
+                            bp = fmaf(qreg[h][e], f16f(km[CPL + e]), bp);
+                        }
+                        float *dstq = qp + (h * 4 + pcs) * W::QPS + pL0;
+#pragma unroll
+                        for (int e = 0; e < CPL; e += 2) *(float2 *)(dstq + e) = make_float2(qv[e], qv[e + 1]);
+                        bias[h] = warp_sum(bp);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < CPL; ++e)
+                        sz[pcs * (D / 4) + pL0 + e] = make_float2(f16f(km[e]), f16f(km[CPL + e]));
+                }
+                __syncwarp();
+
+                // Keys: lane (tq, cs) scores tokens 4tq..4tq+3 over slice cs.
+                uint32_t kw[L::WPL];
+#pragma unroll
+                for (int c = 0; c < L::WPL / 4; ++c) {
+                    uint4 v4 = *(const uint4 *)(st + L::KC + (c * 32 + lane) * 16);
+                    kw[4 * c] = v4.x;
+                    kw[4 * c + 1] = v4.y;
+                    kw[4 * c + 2] = v4.z;
+                    kw[4 * c + 3] = v4.w;
+                }
+                float part[4][HG];
+                if constexpr (!ROPE) {
+                    float2 acc[4][HG];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+#pragma unroll
+                        for (int h = 0; h < HG; ++h) acc[t][h] = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int k = 0; k < KW; ++k) {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4) {
+                            float4 q4[HG];
+#pragma unroll
+                            for (int h = 0; h < HG; ++h)
+                                q4[h] = *(const float4 *)(qp + (h * 4 + cs) * W::QPS + 16 * k + i);
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const uint32_t w = kw[t * KW + k], w22 = w >> 22;
+                                const float2 c01 = code_pair(w, w22, i);
+                                const float2 c23 = code_pair(w, w22, i + 2);
+#pragma unroll
+                                for (int h = 0; h < HG; ++h) {
+                                    acc[t][h] = ffma2(make_float2(q4[h].x, q4[h].y), c01, acc[t][h]);
+                                    acc[t][h] = ffma2(make_float2(q4[h].z, q4[h].w), c23, acc[t][h]);
+                                }
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+#pragma unroll
+                        for (int h = 0; h < HG; ++h) part[t][h] = acc[t][h].x + acc[t][h].y;
+                } else {
+                    // Dequantize, rotate at absolute positions, dot with q.
+                    const long long tbase = it * kG + 4 * tq;
+#pragma unroll 1
+                    for (int t = 0; t < 4; ++t) {
+                        float kh[D / 4];
+#pragma unroll
+                        for (int k = 0; k < KW; ++k) {
+                            const uint32_t w = kw[t * KW + k], w22 = w >> 22;
+#pragma unroll
+                            for (int i = 0; i < 16; i += 2) {
+                                const float2 c = code_pair(w, w22, i);
+                                const float2 s0 = sz[cs * (D / 4) + 16 * k + i];
+                                const float2 s1 = sz[cs * (D / 4) + 16 * k + i + 1];
+                                kh[16 * k + i] = fmaf(c.x, s0.x, s0.y);
+                                kh[16 * k + i + 1] = fmaf(c.y, s1.x, s1.y);
+                            }
+                        }
+                        const float pos = (float)(tbase + t);
+#pragma unroll
+                        for (int i = 0; i < HALF; ++i) {
+                            const float a = __fmul_rn(pos, __ldg(p.inv_freq + cs * HALF + i));
+                            float sn, cn;
+                            sincosf(a, &sn, &cn);
+                            const float x = kh[i], y = kh[HALF + i];
+                            kh[i] = x * cn - y * sn;
+                            kh[HALF + i] = y * cn + x * sn;
+                        }
+#pragma unroll
+                        for (int h = 0; h < HG; ++h) {
+                            float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+                            for (int i = 0; i < HALF; ++i) {
+                                d0 = fmaf(qs[h * D + cs * HALF + i], kh[i], d0);
+                                d1 = fmaf(qs[h * D + D / 2 + cs * HALF + i], kh[HALF + i], d1);
+                            }
+                            part[t][h] = d0 + d1;
+                        }
+                    }
+                }
+                // Transpose-reduce the 4 token partials over the 4 slices: lane
+                // (tq, cs) ends with token 4tq + cs = lane.
+                float sc[HG];
+#pragma unroll
+                for (int h = 0; h < HG; ++h) {
+                    const bool hiB = cs & 2, loB = cs & 1;
+                    float send0 = hiB ? part[0][h] : part[2][h];
+                    float send1 = hiB ? part[1][h] : part[3][h];
+                    float k0 = (hiB ? part[2][h] : part[0][h]) + __shfl_xor_sync(FULL, send0, 2);
+                    float k1 = (hiB ? part[3][h] : part[1][h]) + __shfl_xor_sync(FULL, send1, 2);
+                    float send = loB ? k0 : k1;
+                    float keep = (loB ? k1 : k0) + __shfl_xor_sync(FULL, send, 1);
+                    sc[h] = ROPE ? keep : keep + bias[h];
+                }
+                float pr[HG];
+                softmax_step(sc, pr, true);
+
+                // Value scales for token `lane`.
+                const uint16_t *vm = (const uint16_t *)(st + L::VM + lane * (D / 8));
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    const float svj = f16f(vm[j]), zvj = f16f(vm[NJ + j]);
+#pragma unroll
+                    for (int h = 0; h < HG; ++h) {
+                        pp[(h * NJ + j) * W::PPS + lane] = pr[h] * svj;
+                        zacc[h][j] = fmaf(pr[h], zvj, zacc[h][j]);
+                    }
+                }
+                __syncwarp();
+
+                // Values: lane owns channels [lane*CPL, (lane+1)*CPL).
+                uint32_t vw[L::WPL];
+#pragma unroll
+                for (int c = 0; c < L::WPL / 4; ++c) {
+                    uint4 v4 = *(const uint4 *)(st + L::VC + (c * 32 + lane) * 16);
+                    vw[4 * c] = v4.x;
+                    vw[4 * c + 1] = v4.y;
+                    vw[4 * c + 2] = v4.z;
+                    vw[4 * c + 3] = v4.w;
+                }
+#pragma unroll
+                for (int u = 0; u < L::WPL; ++u) {
+                    const uint32_t w = vw[u], w22 = w >> 22;
+#pragma unroll
+                    for (int t4 = 0; t4 < L::TPW; t4 += 4) {
+                        float4 p4[HG];
+#pragma unroll
+                        for (int h = 0; h < HG; ++h)
+                            p4[h] = *(const float4 *)(pp + (h * NJ + jl) * W::PPS + u * L::TPW + t4);
+#pragma unroll
+                        for (int tt = 0; tt < 4; ++tt) {
+#pragma unroll
+                            for (int c = 0; c < CPL; c += 2) {
+                                const float2 cc = code_pair(w, w22, (t4 + tt) * CPL + c);
+#pragma unroll
+                                for (int h = 0; h < HG; ++h) {
+                                    const float pv = tt == 0 ? p4[h].x : tt == 1 ? p4[h].y : tt == 2 ? p4[h].z : p4[h].w;
+                                    accV[h][c / 2] = ffma2(make_float2(pv, pv), cc, accV[h][c / 2]);
+                                }
+                            }
+                        }
+                    }
+                }
+            } else {
+                // ---------------- residual slice of up to 6 tokens ----------------
+                const int t0 = (int)(it - p.n_groups) * kResTok;
+                const int nt = min(kResTok, p.r - t0);
+                const uint16_t *rk = (const uint16_t *)st;
+                const uint16_t *rv = (const uint16_t *)(st + kResTok * D * 2);
+                const bool valid = tq < nt;
+                float sc[HG];
+                {
+                    float kx[2][HALF];
+                    if (valid) {
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            const uint16_t *src = rk + tq * D + half * (D / 2) + cs * HALF;
+#pragma unroll
+                            for (int i = 0; i < HALF; i += 8) {
+                                uint4 v4 = *(const uint4 *)(src + i);
+                                const uint16_t *e = (const uint16_t *)&v4;
+#pragma unroll
+                                for (int z = 0; z < 8; ++z) kx[half][i + z] = to_f<DT>(e[z]);
+                            }
+                        }
+                        if constexpr (ROPE) {
+                            const float pos = (float)(p.n_q + t0 + tq);
+#pragma unroll
+                            for (int i = 0; i < HALF; ++i) {
+                                const float a = __fmul_rn(pos, __ldg(p.inv_freq + cs * HALF + i));
+                                float sn, cn;
+                                sincosf(a, &sn, &cn);
+                                const float x = kx[0][i], y = kx[1][i];
+                                kx[0][i] = x * cn - y * sn;
+                                kx[1][i] = y * cn + x * sn;
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int half = 0; half < 2; ++half)
+#pragma unroll
+                            for (int i = 0; i < HALF; ++i) kx[half][i] = 0.f;
+                    }
+#pragma unroll
+                    for (int h = 0; h < HG; ++h) {
+                        float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+                        for (int i = 0; i < HALF; ++i) {
+                            d0 = fmaf(qs[h * D + cs * HALF + i], kx[0][i], d0);
+                            d1 = fmaf(qs[h * D + D / 2 + cs * HALF + i], kx[1][i], d1);
+                        }
+                        float d = d0 + d1;
+                        d += __shfl_xor_sync(FULL, d, 1);
+                        d += __shfl_xor_sync(FULL, d, 2);
+                        sc[h] = valid ? d : -INFINITY;
+                    }
+                }
+                float pr[HG];
+                softmax_step(sc, pr, valid && cs == 0);
+                for (int t = 0; t < nt; ++t) {
+                    const uint16_t *vrow = rv + t * D + lane * CPL;
+                    float vx[CPL];
+#pragma unroll
+                    for (int c = 0; c < CPL; ++c) vx[c] = to_f<DT>(vrow[c]);
+#pragma unroll
+                    for (int h = 0; h < HG; ++h) {
+                        const float pt = __shfl_sync(FULL, pr[h], 4 * t);
+#pragma unroll
+                        for (int c = 0; c < CPL; c += 2)
+                            accV[h][c / 2] = ffma2(make_float2(pt, pt), make_float2(vx[c], vx[c + 1]),
+                                                   accV[h][c / 2]);
+                    }
+                }
+            }
+            // Stage consumed: refill it with the item kStages ahead.
+            __syncwarp();
+            ++consumed;
+            issue_next();
+        }
+        if (failed) break;
+
+        // ---------------- this warp's partial for sequence s ----------------
+        const long long first = sp.owner(s * sp.C);
+        const long long last = sp.owner((s + 1) * sp.C - 1);
+        const int count = (int)(last - first + 1);
+        const int slot = (int)(gw - first);
+        float lt[HG], zt[HG][NJ];
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+            lt[h] = warp_sum(lsum[h]);
+#pragma unroll
+            for (int j = 0; j < NJ; ++j) zt[h][j] = warp_sum(zacc[h][j]);
+        }
+        float *outrow = p.out + (b * p.H_q + (long long)hk * HG) * D;
+        if (count == 1) {
+#pragma unroll
+            for (int h = 0; h < HG; ++h) {
+                const float inv = 1.0f / lt[h];
+#pragma unroll
+                for (int c = 0; c < CPL; c += 2) {
+                    const float2 o = accV[h][c / 2];
+                    *(float2 *)(outrow + h * D + lane * CPL + c) =
+                        make_float2((o.x + zt[h][jl]) * inv, (o.y + zt[h][jl]) * inv);
+                }
+            }
+            continue;
+        }
+        float *pbase = p.partials + ((s * p.slots) * HG) * (long long)PSTRIDE;
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+            float *pr = pbase + ((long long)slot * HG + h) * PSTRIDE;
+#pragma unroll
+            for (int c = 0; c < CPL; c += 2) {
+                const float2 o = accV[h][c / 2];
+                *(float2 *)(pr + lane * CPL + c) = make_float2(o.x + zt[h][jl], o.y + zt[h][jl]);
+            }
+            if (lane == 0) *(float2 *)(pr + D) = make_float2(m[h], lt[h]);
+        }
+        __syncwarp();
+        int is_last = 0;
+        if (lane == 0) {
+            __threadfence();
+            is_last = atomicAdd(p.tickets + s, 1) == count - 1;
+        }
+        is_last = __shfl_sync(FULL, is_last, 0);
+        if (!is_last) continue;
+        __threadfence();
+        // Log-sum-exp merge of the `count` partials of sequence s.
+#pragma unroll 1
+        for (int h = 0; h < HG; ++h) {
+            float mx = -INFINITY;
+            for (int k = lane; k < count; k += 32)
+                mx = fmaxf(mx, __ldcg(pbase + ((long long)k * HG + h) * PSTRIDE + D));
+            mx = warp_max(mx);
+            float lacc = 0.f;
+            float o[CPL];
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) o[c] = 0.f;
+#pragma unroll 4
+            for (int k = 0; k < count; ++k) {
+                const float *pk = pbase + ((long long)k * HG + h) * PSTRIDE;
+                const float2 ml = __ldcg((const float2 *)(pk + D));
+                const float wgt = ex2(ml.x - mx);
+                lacc = fmaf(wgt, ml.y, lacc);
+#pragma unroll
+                for (int c = 0; c < CPL; c += 2) {
+                    const float2 v = __ldcg((const float2 *)(pk + lane * CPL + c));
+                    o[c] = fmaf(wgt, v.x, o[c]);
+                    o[c + 1] = fmaf(wgt, v.y, o[c + 1]);
+                }
+            }
+            const float inv = 1.0f / lacc;
+#pragma unroll
+            for (int c = 0; c < CPL; c += 2)
+                *(float2 *)(outrow + h * D + lane * CPL + c) = make_float2(o[c] * inv, o[c + 1] * inv);
+        }
+        if (lane == 0) p.tickets[s] = 0;
+    }
+
+    if (failed) {
+        if (lane == 0) atomicCAS(p.err, 0, kErrWaitTimeout);
+        // Let the copies already in flight land before the warp leaves.
+        while (consumed < issued) {
+            wait_stage(consumed);
+            ++consumed;
+        }
+    }
+}
+
+template <int D, int HG, bool ROPE>
+static int warps_per_cta()
+{
+    return DecodeShape<D, HG, ROPE>::NW;
+}
+
+int decode_warps_per_cta(int D, int HG, int pre_rope)
+{
+#define KIVI_NW(DD, HH)                                                            \
+    if (D == DD && HG == HH) return pre_rope ? warps_per_cta<DD, HH, true>()        \
+                                             : warps_per_cta<DD, HH, false>();
+    KIVI_NW(64, 1) KIVI_NW(64, 2) KIVI_NW(64, 4) KIVI_NW(64, 8)
+    KIVI_NW(128, 1) KIVI_NW(128, 2) KIVI_NW(128, 4) KIVI_NW(128, 8)
+#undef KIVI_NW
+    return 0;
+}
+
+template <int D, int HG, int DT, bool ROPE>
+static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t st)
+{
+    using S = DecodeShape<D, HG, ROPE>;
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
+        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, HG, DT, ROPE>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+        if (e != cudaSuccess) return e;
+        configured_dev = dev;
+    }
+    const long long grid = (p.warps + S::NW - 1) / S::NW;
+    decode_kernel<D, HG, DT, ROPE><<<(unsigned)grid, S::NW * 32, S::SMEM, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <int D, int HG>
+static cudaError_t launch_decode_hg(int dtype, int pre_rope, const DecodeParams &p, cudaStream_t st)
+{
+    if (dtype) {
+        return pre_rope ? launch_decode_t<D, HG, 1, true>(p, st) : launch_decode_t<D, HG, 1, false>(p, st);
+    }
+    return pre_rope ? launch_decode_t<D, HG, 0, true>(p, st) : launch_decode_t<D, HG, 0, false>(p, st);
+}
+
+cudaError_t launch_decode(int D, int HG, int dtype, int pre_rope, const DecodeParams &p,
+                          cudaStream_t st)
+{
+#define KIVI_CASE(DD, HH) \
+    if (D == DD && HG == HH) return launch_decode_hg<DD, HH>(dtype, pre_rope, p, st);
+    KIVI_CASE(64, 1) KIVI_CASE(64, 2) KIVI_CASE(64, 4) KIVI_CASE(64, 8)
+    KIVI_CASE(128, 1) KIVI_CASE(128, 2) KIVI_CASE(128, 4) KIVI_CASE(128, 8)
+#undef KIVI_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kivi

@@ -1,0 +1,60 @@
+// kivi_internal.h -- kernel launch interface between the C ABI and the CUDA
+// kernels.  Internal to the library.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace kivi {
+
+// Quantize whole groups of 32 tokens into the packed store (prefill and the
+// flush of a full residual), optionally copying the prefill's residual rows and
+// writing an appended token into residual slot 0 after the flush has read it.
+struct QuantParams {
+    const uint16_t *srcK, *srcV;  // rows of source group 0 of sequence 0
+    long long src_seq_rows;       // rows between consecutive sequences in src
+    uint8_t *packed;              // [seqs][ngcap][24*D]
+    long long ngcap;              // group capacity per sequence
+    long long g_dst0;             // destination index of source group 0
+    int n_g;                      // groups per sequence to quantize
+    long long seqs;
+    uint16_t *resK, *resV;        // [seqs][R][D]
+    int R;
+    int r_copy;                   // prefill: residual rows to copy (0: none)
+    long long copy_row0;          // prefill: first source row of the residual
+    const uint16_t *newK, *newV;  // flush: token to store in slot 0 (or null)
+};
+
+struct DecodeParams {
+    const uint8_t *packed;
+    long long ngcap;
+    const uint16_t *resK, *resV;
+    int R;
+    const uint16_t *q;
+    float *out;
+    float *partials;     // [seqs][slots][HG][D+4]
+    int *tickets;        // [seqs]
+    int *err;            // status word
+    int H_kv, H_q;
+    long long seqs;
+    long long n_groups;  // quantized groups per sequence
+    int r;               // residual tokens
+    long long n_q;       // absolute position of residual slot 0
+    int wg, wr;          // split weights of a group / a residual item
+    long long warps;     // total warps of the split (<= total weight)
+    int slots;           // partial slots per sequence
+    float qscale;        // log2(e) / sqrt(D)
+    const float *inv_freq;  // RoPE inverse frequencies [D/2] (pre-RoPE caches)
+};
+
+int num_sms();
+
+cudaError_t launch_quant(int D, int dtype, const QuantParams &p, cudaStream_t st);
+cudaError_t launch_append(int D, const uint16_t *k, const uint16_t *v, uint16_t *resK,
+                          uint16_t *resV, long long seqs, int R, int slot, cudaStream_t st);
+// Warps per CTA of the decode kernel for this shape (0 if unsupported).
+int decode_warps_per_cta(int D, int HG, int pre_rope);
+cudaError_t launch_decode(int D, int HG, int dtype, int pre_rope, const DecodeParams &p,
+                          cudaStream_t st);
+
+}  // namespace kivi

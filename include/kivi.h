@@ -1,0 +1,184 @@
+/*
+ * kivi.h -- C ABI of the B200 (sm_100a) KIVI asymmetric 2-bit KV cache.
+ *
+ * The method (KIVI: A Tuning-Free Asymmetric 2bit Quantization for KV Cache;
+ * "KIVI Quantization Secures Llama-2 Accuracy at Two Bits", paragraphs 1-4;
+ * record kv-efficiency/kivi-2bit-llama2-13b-mha-4k, fields "KV bytes basis"
+ * and "Quant method"):
+ *   - keys are quantized per channel: one (scale, zero) per channel per G
+ *     consecutive tokens; values per token: one (scale, zero) per G
+ *     consecutive channels of a token; 2-bit codes, zero = group minimum,
+ *     scale = (max - min)/3, code = clamp(rint((x - zero)/scale), 0, 3), with
+ *     scale and zero stored as IEEE fp16 and codes taken against the stored
+ *     values;
+ *   - the newest tokens stay in a full-precision residual of R slots; prefill
+ *     of T tokens quantizes n_q = R*floor((T-1)/R) and keeps r = T - n_q in
+ *     [1, R]; an append into a full residual first quantizes all R residual
+ *     tokens into the grouped store;
+ *   - decode attention softmax(q.k/sqrt(D)) v runs directly over the packed
+ *     cache plus the residual; query head h reads kv head h / (H_q/H_kv);
+ *   - optionally keys are quantized before RoPE (KIVI article, paragraph 4;
+ *     KVQuant summary, "Pre-RoPE Key Quantization") and rotated at dequant:
+ *     rotate-half pairs (i, i+D/2), absolute positions from 0, angle =
+ *     fp32(t * inv_freq_i), inv_freq_i = fp32(theta^(-2i/D)).
+ *
+ * Conventions shared by every call
+ *   - Pointers named K, V, k_t, v_t, q, out are DEVICE pointers owned by the
+ *     caller, 16-byte aligned, contiguous:
+ *       K, V      [B, H_kv, T, D]  cache dtype
+ *       k_t, v_t  [B, H_kv, D]     cache dtype
+ *       q         [B, H_q, D]      cache dtype, already rotated by RoPE
+ *       out       [B, H_q, D]      fp32
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call that launches work is asynchronous on it; calls on
+ *     one cache must be ordered by the caller (one stream per cache).
+ *   - Arguments are checked before any launch; on an error status nothing
+ *     was launched and the cache is unchanged.  KIVI_ERR_CUDA reports a
+ *     launch or runtime failure (cudaGetLastError), after which the cache
+ *     contents are undefined.
+ *   - Sequence lengths live on the host (no device->host synchronisation in
+ *     prefill, append or decode).
+ *   - A cache is not thread-safe.  No call allocates device memory except
+ *     kivi_cache_create / kivi_cache_create_ex without a workspace.
+ */
+#ifndef KIVI_H
+#define KIVI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KIVI_API __attribute__((visibility("default")))
+#else
+#define KIVI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct kivi_cache kivi_cache; /* opaque; one per layer */
+
+typedef enum { KIVI_F16 = 0, KIVI_BF16 = 1 } kivi_dtype;
+
+typedef enum {
+    KIVI_OK = 0,
+    KIVI_ERR_ARG = 1,         /* bad pointer, size or alignment */
+    KIVI_ERR_UNSUPPORTED = 2, /* valid but not built (e.g. D not in {64,128}) */
+    KIVI_ERR_CAPACITY = 3,    /* would exceed T_max tokens */
+    KIVI_ERR_STATE = 4,       /* prefill twice, decode/append before prefill */
+    KIVI_ERR_OOM = 5,         /* device allocation failed / workspace too small */
+    KIVI_ERR_CUDA = 6,        /* CUDA runtime or launch error */
+    KIVI_ERR_DEVICE = 7       /* a kernel reported a failed bounded wait */
+} kivi_status;
+
+/*
+ * Cache geometry.  Supported: D in {64, 128}, G == 32, R a positive multiple
+ * of G, dtype KIVI_F16 or KIVI_BF16, 1 <= T_max.  T_max bounds the total
+ * number of tokens (prefill plus appends).  pre_rope != 0 stores keys before
+ * RoPE and rotates them in decode with base rope_theta (e.g. 10000).
+ * workspace: optional caller-owned device memory of at least
+ * kivi_cache_required_bytes(cfg) bytes, 256-byte aligned, which then holds
+ * every device buffer of the cache (the library allocates nothing); it must
+ * outlive the cache.
+ */
+typedef struct {
+    int B, H_kv, D, G, R;
+    kivi_dtype dtype;
+    long long T_max;
+    int pre_rope;
+    float rope_theta;
+    void *workspace;
+    size_t workspace_bytes;
+} kivi_config;
+
+/* Device bytes of a cache, by purpose (allocated capacity). */
+typedef struct {
+    size_t codes;    /* 2-bit K and V codes for ceil(T_max/G)*G tokens */
+    size_t meta;     /* fp16 scale and zero of every K and V group */
+    size_t residual; /* R slots of K and V in the cache dtype */
+    size_t scratch;  /* decode partials, tickets, status word, RoPE table */
+    size_t total;    /* all of the above, with alignment padding */
+} kivi_bytes;
+
+/* Library version of this ABI (bumped on incompatible changes). */
+KIVI_API int kivi_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+KIVI_API const char *kivi_status_string(kivi_status s);
+
+/* Create a cache on the current CUDA device; allocates its device memory with
+ * cudaMalloc.  pre_rope = 0.  *out receives the handle. */
+KIVI_API kivi_status kivi_cache_create(int B, int H_kv, int D, int G, int R, kivi_dtype dtype,
+                                       long long T_max, kivi_cache **out);
+
+/* Create from a full configuration (pre-RoPE keys, caller workspace). */
+KIVI_API kivi_status kivi_cache_create_ex(const kivi_config *cfg, kivi_cache **out);
+
+/* Device bytes needed for cfg (ignores cfg->workspace). */
+KIVI_API kivi_status kivi_cache_required_bytes(const kivi_config *cfg, size_t *bytes);
+
+/* Quantize the first n_q = R*floor((T-1)/R) tokens of K, V into the grouped
+ * store and copy the last r = T - n_q tokens into the residual.
+ * 1 <= T <= T_max; KIVI_ERR_STATE if already prefilled (see kivi_cache_reset). */
+KIVI_API kivi_status kivi_prefill(kivi_cache *c, const void *K, const void *V, long long T,
+                         void *stream);
+
+/* Append one token per (batch, kv head).  If the residual holds R tokens they
+ * are first quantized as tokens [n_q, n_q+R) (n_q += R, r = 0); the token then
+ * goes to residual slot r (r += 1).  KIVI_ERR_CAPACITY past T_max tokens. */
+KIVI_API kivi_status kivi_append(kivi_cache *c, const void *k_t, const void *v_t, void *stream);
+
+/* Decode attention of one query per head over all n_q + r tokens.
+ * H_q a multiple of H_kv with H_q/H_kv in {1, 2, 4, 8}.  out is fp32. */
+KIVI_API kivi_status kivi_decode_attn(kivi_cache *c, const void *q, int H_q, float *out,
+                             void *stream);
+
+/* Forget the cached tokens (host counters only; device buffers are kept). */
+KIVI_API kivi_status kivi_cache_reset(kivi_cache *c);
+
+/* Current split: n_q quantized tokens, r residual tokens. */
+KIVI_API kivi_status kivi_cache_length(const kivi_cache *c, long long *n_q, int *r);
+
+/* Allocated device bytes of the cache, by purpose. */
+KIVI_API kivi_status kivi_cache_bytes(const kivi_cache *c, kivi_bytes *out);
+
+/*
+ * Copy sequences [seq0, seq0 + nseq) of the cache (sequence = b*H_kv + h) to
+ * HOST arrays in the canonical unpacked layout (testing and inspection;
+ * synchronises the device).  Arrays are caller-owned host memory:
+ *   codesK, codesV [nseq, n_q, D]   uint8 in {0..3}
+ *   sK, zK         [nseq, n_q/G, D] fp16 bits
+ *   sV, zV         [nseq, n_q, D/G] fp16 bits
+ *   resK, resV     [nseq, r, D]     cache dtype
+ * Any array pointer may be NULL to skip it.
+ */
+KIVI_API kivi_status kivi_export(const kivi_cache *c, long long seq0, long long nseq,
+                                 uint8_t *codesK, uint8_t *codesV, uint16_t *sK, uint16_t *zK,
+                                 uint16_t *sV, uint16_t *zV, void *resK, void *resV);
+
+/* Read (synchronously) and clear the cache's device status word: 0 if every
+ * bounded wait in its kernels completed, else the code of the first failure. */
+KIVI_API kivi_status kivi_device_status(kivi_cache *c, int *code);
+
+/* Release the cache (frees its memory unless it lives in a caller workspace). */
+KIVI_API kivi_status kivi_cache_destroy(kivi_cache *c);
+
+/*
+ * Host-side view of the decode work split, for inspection and tests; needs no
+ * GPU.  The flattened work of all B*H_kv sequences (n_groups quantized groups
+ * and ceil(r/6) residual items of up to 6 tokens each, weighted wg and wr) is
+ * cut into `warps` equal contiguous ranges.  For sequence `seq` it reports
+ * out[0] = first warp, out[1] = last warp (inclusive), and for warp `warp`
+ * out[2], out[3] = the half-open item range it owns in that sequence
+ * (empty if out[2] == out[3]).
+ */
+KIVI_API kivi_status kivi_decode_split(long long seqs, long long n_groups, int r, int wg, int wr,
+                              long long warps, long long seq, long long warp,
+                              long long out[4]);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KIVI_H */

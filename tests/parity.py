@@ -1,0 +1,122 @@
+"""Helpers shared by the GPU parity tests: drive the CUDA library and the CPU
+oracle on the same seeded inputs and compare them.
+
+Bars: codes, scales, zeros and residual rows bit-exact; attention output with
+relative L2 error <= 5e-3 and max-abs error <= 2e-3 * max|ref| against the
+oracle's double-precision attention over the same dequantized cache.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from bit_asymmetric_kv_prefill_b200 import KiviCache, synth
+
+REL_L2 = 5e-3
+MAX_ABS = 2e-3
+
+
+def odtype(w):
+    return oracle.DTYPE_BF16 if w.dtype == "bf16" else oracle.DTYPE_F16
+
+
+def attn_errors(out, ref):
+    out = np.asarray(out, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rel = np.linalg.norm(out - ref) / max(np.linalg.norm(ref), 1e-30)
+    mabs = np.abs(out - ref).max() / max(np.abs(ref).max(), 1e-30)
+    return rel, mabs
+
+
+def assert_attn_close(out, ref, what=""):
+    assert np.all(np.isfinite(out)), what
+    rel, mabs = attn_errors(out, ref)
+    assert rel <= REL_L2 and mabs <= MAX_ABS, f"{what}: rel-L2 {rel:.3e}, max-abs/max {mabs:.3e}"
+    return rel, mabs
+
+
+def assert_store_equal(cache: KiviCache, orc: oracle.OracleCache, seqs):
+    """Bit-exact comparison of the quantized store and residual of the given
+    flattened sequences (b*H_kv + h) of the GPU cache with an oracle cache that
+    holds every sequence."""
+    assert cache.length() == (orc.n_q, orc.r)
+    ref = orc.quantized()
+    for s in seqs:
+        got = cache.export(s, 1)
+        ob, oh = divmod(s, orc.H)
+        for key in ("codesK", "codesV", "sK", "zK", "sV", "zV", "resK", "resV"):
+            a, b = got[key][0], ref[key][ob, oh]
+            if not np.array_equal(a, b):
+                bad = np.argwhere(a != b)
+                raise AssertionError(f"{key} differs for sequence {s} at {bad[:5].tolist()} "
+                                     f"({len(bad)} entries): gpu {a[tuple(bad[0])]} "
+                                     f"oracle {b[tuple(bad[0])]}")
+
+
+class Pair:
+    """A GPU cache and an oracle cache fed identical bits.  The oracle holds
+    either every sequence or only the sampled ones (`sample`)."""
+
+    def __init__(self, w: synth.Workload, seed=0, sample=None, T_max=None):
+        self.w = w
+        self.seed = seed
+        self.HG = w.H_q // w.H_kv
+        self.cache = KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype,
+                               T_max or w.T_max, pre_rope=w.pre_rope, rope_theta=w.rope_theta)
+        self.sample = sample
+        nb, nh = (w.B, w.H_kv) if sample is None else (len(sample), 1)
+        self.orc = oracle.OracleCache(nb, nh, w.D, w.G, w.R, odtype(w), T_max or w.T_max,
+                                      pre_rope=w.pre_rope, rope_theta=w.rope_theta)
+
+    def seqs(self):
+        return list(range(self.w.B * self.w.H_kv)) if self.sample is None else list(self.sample)
+
+    def _pick(self, t: torch.Tensor):
+        """[B, H_kv, ...] -> host bits of the oracle's sequences."""
+        if self.sample is None:
+            return synth.bits(t)
+        rows = [t[s // self.w.H_kv, s % self.w.H_kv] for s in self.sample]
+        return synth.bits(torch.stack(rows)[:, None])
+
+    def _pick_q(self, q: torch.Tensor):
+        if self.sample is None:
+            return synth.bits(q)
+        HG = self.HG
+        rows = [q[s // self.w.H_kv, (s % self.w.H_kv) * HG:(s % self.w.H_kv + 1) * HG] for s in self.sample]
+        return synth.bits(torch.stack(rows))
+
+    def prefill(self, K, V):
+        self.cache.prefill(K, V)
+        self.orc.prefill(self._pick(K), self._pick(V))
+
+    def append(self, k, v):
+        self.cache.append(k, v)
+        self.orc.append(self._pick(k), self._pick(v))
+
+    def decode(self, q):
+        """GPU output restricted to the oracle's sequences, and the oracle's."""
+        out = self.cache.decode(q)
+        torch.cuda.synchronize()
+        ref = self.orc.decode(self._pick_q(q))
+        o = out.cpu().numpy()
+        if self.sample is None:
+            return o, ref
+        HG = self.HG
+        got = np.stack([o[s // self.w.H_kv, (s % self.w.H_kv) * HG:(s % self.w.H_kv + 1) * HG]
+                        for s in self.sample])
+        return got, ref
+
+    def check_store(self, every=1):
+        seqs = self.seqs()[::every]
+        if self.sample is None:
+            assert_store_equal(self.cache, self.orc, seqs)
+        else:
+            # oracle sequence i <-> GPU sequence sample[i]
+            assert self.cache.length() == (self.orc.n_q, self.orc.r)
+            ref = self.orc.quantized()
+            for i, s in enumerate(self.sample):
+                got = self.cache.export(s, 1)
+                for key in ref:
+                    if not np.array_equal(got[key][0], ref[key][i, 0]):
+                        raise AssertionError(f"{key} differs for sequence {s}")

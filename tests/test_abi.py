@@ -1,0 +1,108 @@
+"""CPU checks of the C-ABI library: it loads, exports every declared symbol,
+rejects bad configurations before touching the GPU, and its decode work split
+covers every item exactly once."""
+import ctypes
+import itertools
+import subprocess
+
+import pytest
+
+import bit_asymmetric_kv_prefill_b200 as kivi
+from bit_asymmetric_kv_prefill_b200 import build as kbuild
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    kbuild.build()
+
+
+def test_every_declared_symbol_is_exported():
+    declared = kivi.declared_symbols()
+    assert len(declared) >= 14
+    nm = subprocess.run(["nm", "-D", "--defined-only", kivi.LIB_PATH], capture_output=True,
+                        text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in nm.splitlines() if " T " in ln}
+    missing = [s for s in declared if s not in exported]
+    assert not missing, missing
+    L = kivi.lib()
+    for s in declared:
+        assert getattr(L, s) is not None
+
+
+def test_status_strings_and_version():
+    assert kivi.abi_version() == 1
+    names = {kivi.status_string(c) for c in range(8)}
+    assert len(names) == 8 and "ok" in names
+    assert kivi.status_string(99) == "unknown status"
+
+
+def _cfg(**kw):
+    base = dict(B=1, H_kv=2, D=64, G=32, R=128, dtype=kivi.KIVI_F16, T_max=256, pre_rope=0,
+                rope_theta=10000.0, workspace=None, workspace_bytes=0)
+    base.update(kw)
+    return kivi._Config(*[base[f] for f, _ in kivi._Config._fields_])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=96), 2),             # head_dim without a kernel
+    (dict(G=16, R=128), 2),      # group size other than 32
+    (dict(R=100), 1),            # residual not a multiple of G
+    (dict(dtype=5), 1),
+    (dict(B=0), 1),
+    (dict(T_max=0), 1),
+    (dict(pre_rope=1, rope_theta=0.0), 1),
+])
+def test_bad_configs_are_rejected_before_any_launch(kw, code):
+    h = ctypes.c_void_p()
+    cfg = _cfg(**kw)
+    assert kivi.lib().kivi_cache_create_ex(ctypes.byref(cfg), ctypes.byref(h)) == code
+    assert not h.value
+    n = ctypes.c_size_t()
+    assert kivi.lib().kivi_cache_required_bytes(ctypes.byref(cfg), ctypes.byref(n)) == code
+
+
+def test_null_handles_are_rejected():
+    L = kivi.lib()
+    assert L.kivi_prefill(None, None, None, 10, None) == 1
+    assert L.kivi_append(None, None, None, None) == 1
+    assert L.kivi_decode_attn(None, None, 2, None, None) == 1
+    assert L.kivi_cache_destroy(None) == 1
+    assert L.kivi_cache_reset(None) == 1
+    assert L.kivi_export(None, 0, 1, *([None] * 8)) == 1
+    assert L.kivi_cache_length(None, None, None) == 1
+
+
+@pytest.mark.parametrize("seqs,n_groups,r,wg,wr,warps", [
+    (1, 4, 128, 4, 3, 26),        # tiny workload: 4 groups + 22 residual items
+    (256, 128, 1, 4, 3, 2368),    # Llama-2-7B layer after the first flush
+    (256, 124, 128, 4, 3, 2368),
+    (8, 4092, 128, 4, 3, 2072),   # long context
+    (3, 0, 7, 4, 3, 2),           # residual only
+    (5, 3, 6, 1, 1, 40),
+    (7, 9, 13, 5, 2, 11),
+])
+def test_decode_split_covers_every_item_once(seqs, n_groups, r, wg, wr, warps):
+    n_items = n_groups + -(-r // 6)
+    total = seqs * (n_groups * wg + -(-r // 6) * wr)
+    warps = min(warps, total)
+    for s in range(seqs):
+        first, last, _, _ = kivi.decode_split(seqs, n_groups, r, wg, wr, warps, s, 0)
+        assert 0 <= first <= last < warps
+        covered = []
+        for w in range(warps):
+            f2, l2, i0, i1 = kivi.decode_split(seqs, n_groups, r, wg, wr, warps, s, w)
+            assert (f2, l2) == (first, last)
+            if w < first or w > last:
+                assert i0 == i1, (s, w)
+            covered.extend(range(i0, i1))
+        assert covered == list(range(n_items)), s
+
+
+def test_decode_split_balances_weight():
+    seqs, n_groups, r, wg, wr, warps = 256, 128, 64, 4, 3, 2368
+    load = [0] * warps
+    for s, w in itertools.product(range(0, seqs, 17), range(warps)):
+        _, _, i0, i1 = kivi.decode_split(seqs, n_groups, r, wg, wr, warps, s, w)
+        load[w] += sum(wg if i < n_groups else wr for i in range(i0, i1))
+    per_seq = n_groups * wg + -(-r // 6) * wr
+    assert sum(load) == per_seq * len(range(0, seqs, 17))
