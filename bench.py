@@ -1,0 +1,471 @@
+"""Benchmark: KIVI 2-bit KV cache hot path on B200.
+
+One step = one pass of the whole hot path over the Llama-2-7B layer workload
+(batch 8, 32 MHA heads, head_dim 128, 4,096-token context, G=32, R=128, bf16):
+prefill quantization, then 64 decode steps each appending one token (the first
+append flushes the full residual) and running decode attention.  The step runs
+over `--layers` independent layer caches (default 8) visited round-robin, as a
+model's decode does, so the working set (~1.1 GB) is far larger than the
+126 MB L2 and every decode streams its cache from HBM.
+
+Metric: decode-attention KV tokens x heads per second (sum over decode calls of
+B * H_kv * tokens attended), whole step time in the denominator (prefill and
+appends included).  The decode kernel's achieved HBM bandwidth (algorithmic
+bytes / CUDA-event duration of each launch) is reported against the measured
+copy bandwidth in MEASURED_PEAKS.json.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica
+(no data exchange: sequences and heads are independent) and the reported value
+is the sum over ranks divided by the slowest rank's time.  `--impl reference`
+times the plain CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn KV tokens·heads/s and achieved HBM GB/s vs 8 TB/s"
+UNIT = "KV tokens·heads/s"
+WORKLOAD = "llama2_7b_layer"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_llama2_7b_layer_traffic.json")
+DECODE_SOURCES = ["bit_asymmetric_kv_prefill_b200/csrc/kivi_decode.cu",
+                  "bit_asymmetric_kv_prefill_b200/csrc/kivi_common.cuh"]
+
+
+# ---- workload arithmetic (bytes and units, no method math) ---------------------
+
+def decode_schedule(w):
+    """(n_q, r) seen by each decode call of one layer's step, in order."""
+    R, T = w.R, w.T
+    n_q = R * ((T - 1) // R)
+    r = T - n_q
+    out = []
+    for _ in range(w.steps):
+        if r == R:
+            n_q += R
+            r = 0
+        r += 1
+        out.append((n_q, r))
+    return out
+
+
+def decode_bytes(w, n_q, r):
+    """Algorithmic HBM bytes of one decode call: per quantized (token, kv head)
+    the 2-bit K and V codes plus fp16 scale/zero (D/4 + 4D/G for each of K and
+    V), per residual token 2*D*2 bytes, plus q (bf16) and out (fp32)."""
+    per_q = 2 * (w.D // 4 + 4 * w.D // w.G)
+    per_r = 2 * w.D * 2
+    return w.B * w.H_kv * (n_q * per_q + r * per_r) + w.B * w.H_q * w.D * (2 + 4)
+
+
+def decode_units(w, n_q, r):
+    return w.B * w.H_kv * (n_q + r)
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def traffic_per_launch():
+    """dram read+write bytes per decode launch from the committed ncu summary,
+    or None when absent or taken on other kernel sources."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_source_sha256") != source_hash():
+        return None
+    return d.get("traffic_bytes_per_launch")
+
+
+# ---- clocks ----------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi samples of one GPU during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_key: str):
+        self.bus = bus_key
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu=pci.bus_id,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    @staticmethod
+    def _bus_key(bus: str) -> str:
+        # nvidia-smi's "00000000:1B:00.0" -> "1b:00.0"
+        return bus.strip().lower().split(":", 1)[-1]
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        want = self.bus
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9 or self._bus_key(parts[0]) != want:
+                continue
+            parts = parts[1:]
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---- multi-rank helpers ------------------------------------------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), \
+        int(os.environ.get("LOCAL_RANK", 0))
+
+
+def reduce_max(x: float, device) -> float:
+    """Max of a scalar over ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+    if device.type == "cuda":
+        torch.cuda.synchronize(device)
+
+
+# ---- CPU oracle leg ------------------------------------------------------------------
+
+def oracle_stream_rate(w, seconds: float, max_seqs: int = 1 << 30):
+    """Time the oracle on whole per-sequence streams (prefill + `steps` x
+    (append + decode)) of the workload until `seconds` elapse; returns
+    (units/s, sequences done, seconds)."""
+    import oracle
+    from bit_asymmetric_kv_prefill_b200 import synth
+    sched = decode_schedule(w)
+    units_seq = sum(n_q + r for n_q, r in sched)
+    one = synth.scaled(w, B=1, H_q=w.H_q // w.H_kv, H_kv=1)
+    done, t_used = 0, 0.0
+    dt = oracle.DTYPE_BF16 if w.dtype == "bf16" else oracle.DTYPE_F16
+    while (t_used < seconds or done == 0) and done < max_seqs:
+        K, V = synth.prefill_inputs(one, seed=done)
+        kb, vb = synth.bits(K), synth.bits(V)
+        steps = [tuple(synth.bits(x) for x in synth.step_inputs(one, s, seed=done))
+                 for s in range(1, w.steps + 1)]
+        c = oracle.OracleCache(1, 1, w.D, w.G, w.R, dt, w.T_max)
+        t0 = time.perf_counter()
+        c.prefill(kb, vb)
+        for k, v, q in steps:
+            c.append(k, v)
+            c.decode(q)
+        t_used += time.perf_counter() - t0
+        done += 1
+    return units_seq * done / t_used, done, t_used
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    from bit_asymmetric_kv_prefill_b200 import synth
+    oracle.build()
+    w = synth.WORKLOADS[WORKLOAD]
+    for _ in range(args.warmup):
+        oracle_stream_rate(w, 0.0, max_seqs=1)
+    t_total, units_total = 0.0, 0.0
+    units_seq = sum(n_q + r for n_q, r in decode_schedule(w))
+    for _ in range(args.steps):
+        _, n, t = oracle_stream_rate(w, 0.0, max_seqs=1)
+        t_total += t
+        units_total += units_seq * n
+    value = units_total / t_total
+    sample = (f"each step: one (batch, head) sequence of {WORKLOAD}: prefill T={w.T} + "
+              f"{w.steps} x (append + decode), single thread")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, args),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- GPU leg ----------------------------------------------------------------------------
+
+def workload_config(w, args):
+    return {"workload": f"{WORKLOAD}: Llama-2-7B layer shape, batch {w.B}, {w.H_q} MHA heads, "
+                        f"head_dim {w.D}, context {w.T}, G={w.G}, R={w.R}, bf16 input/residual, "
+                        f"prefill + {w.steps} x (append + decode) per layer",
+            "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "D": w.D, "T": w.T, "G": w.G, "R": w.R,
+            "decode_steps": w.steps, "layers_round_robin": args.layers,
+            "l2": f"inputs larger than L2: {args.layers} layer caches visited round-robin "
+                  f"(~{args.layers * 134} MB working set vs 126 MB L2), no explicit flush",
+            "parallelism": f"replicas x{max(1, args.gpus)} (no data-path collective)"}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    import bit_asymmetric_kv_prefill_b200 as kivi
+    from bit_asymmetric_kv_prefill_b200 import KiviCache, synth
+    from bit_asymmetric_kv_prefill_b200 import build as kbuild
+    kbuild.build()
+    L = kivi.lib()
+
+    w = synth.WORKLOADS[WORKLOAD]
+    nl = args.layers
+    sched = decode_schedule(w)
+    bytes_step = sum(decode_bytes(w, n, r) for n, r in sched) * nl
+    units_step = sum(decode_units(w, n, r) for n, r in sched) * nl
+    launches_step = nl * (1 + 2 * w.steps)
+
+    caches = [KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, w.T_max) for _ in range(nl)]
+    Ks, Vs = [], []
+    for l in range(nl):
+        K, V = synth.prefill_inputs(w, seed=1000 * rank + l, device=dev)
+        Ks.append(K)
+        Vs.append(V)
+    steps = [[synth.step_inputs(w, s, seed=1000 * rank + l, device=dev) for l in range(nl)]
+             for s in range(1, w.steps + 1)]
+    outs = [torch.empty(w.B, w.H_q, w.D, dtype=torch.float32, device=dev) for _ in range(nl)]
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    H = [c._h for c in caches]
+    Kp = [ctypes.c_void_p(t.data_ptr()) for t in Ks]
+    Vp = [ctypes.c_void_p(t.data_ptr()) for t in Vs]
+    Sp = [[tuple(ctypes.c_void_p(t.data_ptr()) for t in st) for st in row] for row in steps]
+    Op = [ctypes.c_void_p(o.data_ptr()) for o in outs]
+    T, Hq = w.T, w.H_q
+    reset, prefill, append, decode = (L.kivi_cache_reset, L.kivi_prefill, L.kivi_append,
+                                      L.kivi_decode_attn)
+
+    def one_step(ev=None):
+        bad = 0
+        for l in range(nl):
+            bad |= reset(H[l])
+            bad |= prefill(H[l], Kp[l], Vp[l], T, sp)
+        i = 0
+        for row in Sp:
+            for l in range(nl):
+                k, v, q = row[l]
+                bad |= append(H[l], k, v, sp)
+                if ev is not None:
+                    ev[i][0].record(stream)
+                bad |= decode(H[l], q, Hq, Op[l], sp)
+                if ev is not None:
+                    ev[i][1].record(stream)
+                i += 1
+        if bad:
+            raise RuntimeError("a KIVI call failed during the benchmark")
+
+    for _ in range(args.warmup):
+        one_step()
+    n_dec = nl * w.steps
+    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+               for _ in range(n_dec)] for _ in range(args.steps)]
+    t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(dev)
+    clocks = ClockSampler(f"{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0")
+    barrier(dev)
+    clocks.start()
+    time.sleep(0.3)  # let the sampler attach before the timed region
+    t0e.record(stream)
+    for k in range(args.steps):
+        one_step(events[k])
+    t1e.record(stream)
+    torch.cuda.synchronize(dev)
+    ck = clocks.stop()
+    barrier(dev)
+    ms_local = t0e.elapsed_time(t1e)
+    dec_ms = [a.elapsed_time(b) for ev in events for a, b in ev]
+    dec_avg_local = sum(dec_ms) / len(dec_ms)
+    status = max(c.device_status() for c in caches)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    ms = reduce_max(ms_local, dev)
+    dec_avg = reduce_max(dec_avg_local, dev)
+    value = world * units_step * args.steps / (ms / 1e3)
+    bytes_per_launch = bytes_step / n_dec
+    achieved = bytes_per_launch / (dec_avg / 1e3) / 1e9
+    peak, peak_kind = measured_peak()
+    traffic = traffic_per_launch()
+
+    e2e = run_e2e(args, w, caches, Ks, Vs, steps, dev, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, nseq, secs = oracle_stream_rate(w, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{nseq} (batch, head) sequences of {WORKLOAD}, each prefill T={w.T} + "
+                         f"{w.steps} x (append + decode); {secs:.1f} s single-threaded"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
+            "data": "synthetic", "config": workload_config(w, args),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                         "kernel": "decode_kernel (kivi_decode_attn)",
+                         "alg_bytes_per_launch": bytes_per_launch,
+                         "frac_of_8TBps": achieved / 8000.0},
+            "decode_attn": {"avg_us": 1e3 * dec_avg, "launches_timed": len(dec_ms),
+                            "tokens_heads_per_s": units_step / nl / w.steps / (dec_avg / 1e3),
+                            "gpu_time_share": sum(dec_ms) / ms_local},
+            "e2e": e2e, "gpu_launches": launches_step * args.steps, "clocks": ck,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    for c in caches:
+        c.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, w, caches, Ks, Vs, steps, dev, world):
+    """Same step through the public API with pinned HOST inputs: the H2D copies
+    of every input and the D2H read of every decode output are timed."""
+    import torch
+    nl = len(caches)
+    hK = [k.cpu().pin_memory() for k in Ks]
+    hV = [v.cpu().pin_memory() for v in Vs]
+    hS = [[tuple(t.cpu().pin_memory() for t in st) for st in row] for row in steps]
+    dK = [torch.empty_like(Ks[0]) for _ in range(2)]
+    dV = [torch.empty_like(Vs[0]) for _ in range(2)]
+    dS = [tuple(torch.empty_like(t) for t in steps[0][0]) for _ in range(nl)]
+    hout = [torch.empty(w.B, w.H_q, w.D, dtype=torch.float32).pin_memory() for _ in range(nl)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for l in range(nl):
+            caches[l].reset()
+            dK[l % 2].copy_(hK[l], non_blocking=True)
+            dV[l % 2].copy_(hV[l], non_blocking=True)
+            caches[l].prefill(dK[l % 2], dV[l % 2])
+        for row in hS:
+            for l in range(nl):
+                k, v, q = (d.copy_(h, non_blocking=True) for d, h in zip(dS[l], row[l]))
+                caches[l].append(k, v)
+                out = caches[l].decode(q)
+                hout[l].copy_(out, non_blocking=True)
+
+    n = max(1, min(args.steps, args.e2e_steps))
+    step()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    ms = reduce_max(a.elapsed_time(b), dev)
+    sched = decode_schedule(w)
+    units = sum(decode_units(w, nq, r) for nq, r in sched) * nl
+    h2d = nl * (2 * Ks[0].numel() * 2 + w.steps * sum(t.numel() * 2 for t in steps[0][0]))
+    d2h = nl * w.steps * w.B * w.H_q * w.D * 4
+    return {"value": world * units * n / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": ms / n}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["kivi", "reference"], default="kivi")
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--e2e-steps", dest="e2e_steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", dest="cpu_seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", dest="no_cpu_baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

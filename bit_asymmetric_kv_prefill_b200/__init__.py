@@ -21,7 +21,8 @@ import re
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkivi_b200.so")
+# KIVI_LIB selects another build of the same library (e.g. a tuning variant).
+LIB_PATH = os.environ.get("KIVI_LIB") or os.path.join(_HERE, "libkivi_b200.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "kivi.h")
 
 KIVI_F16, KIVI_BF16 = 0, 1

@@ -41,14 +41,16 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, extra=(), out: str = LIB,
+          build_dir: str = BUILD_DIR) -> str:
+    """Compile every csrc/*.cu for sm_100a and link `out` (extra: nvcc flags)."""
+    if not force and out == LIB and up_to_date():
         return LIB
-    os.makedirs(BUILD_DIR, exist_ok=True)
+    os.makedirs(build_dir, exist_ok=True)
     objs = []
     procs = []
     for src in sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
@@ -57,13 +59,13 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     failed = [src for p, src in procs if p.wait() != 0]
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(failed))
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    tmp = out + ".tmp.%d" % os.getpid()
     cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-Xlinker", "--exclude-libs,ALL"]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

@@ -18,7 +18,7 @@ using namespace kivi;
 namespace {
 
 constexpr int kAbiVersion = 1;
-constexpr int kMaxWarpsPerCta = 16;  // upper bound over decode shapes
+constexpr int kMaxWarpsPerCta = 32;  // upper bound over decode shapes
 constexpr int kMaxGroupHeads = 8;    // largest H_q/H_kv served
 constexpr size_t kAlign = 256;
 
@@ -361,6 +361,8 @@ kivi_status kivi_decode_attn(kivi_cache *c, const void *q, int H_q, float *out, 
     p.slots = c->plan.slots;
     p.qscale = (float)(1.4426950408889634 / std::sqrt((double)c->cfg.D));
     p.inv_freq = c->inv_freq;
+    p.magic = 0x4B000000u;
+    p.neg_magic = -8388608.0f;
     if (warps / p.seqs + 2 > p.slots) return KIVI_ERR_UNSUPPORTED;
     cudaError_t e = launch_decode(c->cfg.D, HG, c->cfg.dtype, c->cfg.pre_rope, p,
                                   (cudaStream_t)stream);
@@ -399,14 +401,26 @@ void unpack_groups(long long nseq, const std::vector<uint8_t> &blk, long long n_
                     uint32_t kw, vw;
                     std::memcpy(&kw, b + L::KC + code_word_offset(lane, u), 4);
                     std::memcpy(&vw, b + L::VC + code_word_offset(lane, u), 4);
+                    // K word u = tok*KW + k of lane (tq, cs): pair i is local
+                    // channels 16k+2i (bits 2i) and 16k+2i+1 (bits 16+2i).
                     const int tok = u / L::KW, k = u % L::KW;
                     const long long tK = g * kG + 4 * (lane >> 2) + tok;
-                    for (int i = 0; i < 16; ++i) {
-                        const int d = k_channel<D>(lane & 3, 16 * k + i);
-                        if (codesK) codesK[(s * nq + tK) * D + d] = (kw >> (2 * i)) & 3u;
-                        const long long tV = g * kG + u * L::TPW + i / L::CPL;
-                        const int dv = lane * L::CPL + i % L::CPL;
-                        if (codesV) codesV[(s * nq + tV) * D + dv] = (vw >> (2 * i)) & 3u;
+                    // V word u of lane (co, th): pair i is token
+                    // 16th + u*TPW + i/(CPL/2), channels co*CPL + 2*(i%(CPL/2)) + {0,1}.
+                    const int co = lane & 15, th = lane >> 4;
+                    for (int i = 0; i < 8; ++i) {
+                        const int d0 = k_channel<D>(lane & 3, 16 * k + 2 * i);
+                        const int d1 = k_channel<D>(lane & 3, 16 * k + 2 * i + 1);
+                        if (codesK) {
+                            codesK[(s * nq + tK) * D + d0] = (kw >> (2 * i)) & 3u;
+                            codesK[(s * nq + tK) * D + d1] = (kw >> (16 + 2 * i)) & 3u;
+                        }
+                        const long long tV = g * kG + 16 * th + u * L::TPW + i / (L::CPL / 2);
+                        const int dv = co * L::CPL + 2 * (i % (L::CPL / 2));
+                        if (codesV) {
+                            codesV[(s * nq + tV) * D + dv] = (vw >> (2 * i)) & 3u;
+                            codesV[(s * nq + tV) * D + dv + 1] = (vw >> (16 + 2 * i)) & 3u;
+                        }
                     }
                 }
             }

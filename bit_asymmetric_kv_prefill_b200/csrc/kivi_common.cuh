@@ -20,17 +20,22 @@ constexpr int kErrWaitTimeout = 1;
 //   [0,    8D)  Kc  K codes.  Lane l = 4*tq + cs holds tokens 4tq..4tq+3 and
 //                   the D/4 channels of slice cs (D/8 from each RoPE half, so
 //                   that rotate-half partners stay in one lane): D/16 words,
-//                   word u = tok*(D/64) + k, slot i of word u <-> local channel
-//                   L = 16k + i.  Words are stored [u/4][lane][u%4].
+//                   word u = tok*(D/64) + k covers local channels
+//                   L = 16k..16k+15.  Words are stored [u/4][lane][u%4].
 //   [8D,  12D)  Km  K scale/zero per channel, permuted order P = cs*(D/4) + L,
 //                   lane l owns P in [l*D/32, (l+1)*D/32): D/32 fp16 scales
 //                   then D/32 fp16 zeros.
-//   [12D, 20D)  Vc  V codes.  Lane l holds channels [l*D/32, (l+1)*D/32) of
-//                   all 32 tokens: word u covers tokens [u*TPW, (u+1)*TPW),
-//                   slot i <-> (token u*TPW + i/CPL, channel l*CPL + i%CPL).
+//   [12D, 20D)  Vc  V codes.  Lane l = 16*th + co holds the D/16 channels of
+//                   octet co, [co*D/16, (co+1)*D/16), for tokens 16th..16th+15:
+//                   D/16 words, word u covers tokens 16th + u*TPW + [0, TPW).
 //   [20D, 24D)  Vm  V scale/zero per token: D/32 fp16 scales then D/32 zeros.
 //
-// Code slot i of a 32-bit word occupies bits [2i, 2i+1] (16 codes per word).
+// A 32-bit word holds 16 two-bit codes as 8 pairs: pair i has its first code
+// at bits [2i, 2i+1] and its second at bits [16+2i, 17+2i].  In a K word pair
+// i is local channels (16k+2i, 16k+2i+1); in a V word pair i is token
+// 16th + u*TPW + i/(CPL/2), channels co*CPL + 2*(i%(CPL/2)) and the next one.
+// Both halves of a pair sit at the same shift, so a decoder reads the pair from
+// the word and from the word shifted right by 16 with one logic op per code.
 // ---------------------------------------------------------------------------
 template <int D>
 struct Layout {
@@ -44,7 +49,8 @@ struct Layout {
     static constexpr int KW = D / 64;    // K words per token per lane
     static constexpr int HALF = D / 8;   // channels per lane per RoPE half
     static constexpr int SLICE = D / 4;  // K channels per lane
-    static constexpr int CPL = D / 32;   // V channels per lane
+    static constexpr int QPL = D / 32;   // K scale/zero entries per lane
+    static constexpr int CPL = D / 16;   // V channels per lane
     static constexpr int TPW = 16 / CPL; // tokens per V word
     static constexpr int NJ = D / kG;    // value groups per token
 };

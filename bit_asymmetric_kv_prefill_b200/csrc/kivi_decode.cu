@@ -38,8 +38,19 @@
 
 namespace kivi {
 
+// Build-time tuning knobs (defaults are the measured best on B200).
+#ifndef KIVI_DECODE_STAGES
+#define KIVI_DECODE_STAGES 3
+#endif
+#ifndef KIVI_DECODE_MAXW
+#define KIVI_DECODE_MAXW 16
+#endif
+#ifndef KIVI_SCALAR_F32
+#define KIVI_SCALAR_F32 0
+#endif
+
 constexpr unsigned FULL = 0xffffffffu;
-constexpr int kStages = 3;
+constexpr int kStages = KIVI_DECODE_STAGES;
 constexpr float kRescaleSlack = 8.0f;
 constexpr long long kWaitLimit = 1LL << 22;
 
@@ -86,6 +97,9 @@ __device__ __forceinline__ float ex2(float x)
 }
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
 {
+#if KIVI_SCALAR_F32
+    return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+#endif
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
         "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
@@ -96,6 +110,9 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
 }
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
 {
+#if KIVI_SCALAR_F32
+    return make_float2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y));
+#endif
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
         "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -106,26 +123,24 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
 }
 
 // ---- code extraction ---------------------------------------------------------
-// Slot i of a word sits at bits [2i, 2i+1].  Slots 0..10 are read in place,
-// slots 11..15 from the word shifted right by 22.  With the field at bit p of
-// the mantissa and biased exponent 150 - p, the float equals 2^(23-p) + c.
-__device__ __forceinline__ float code_raw(uint32_t w, uint32_t w22, int i)
+// Code pair i of a word (split-pair layout): first code at bits 2i of w,
+// second at bits 2i of w16 = w >> 16.  OR-ing the field into the mantissa of
+// 2^23 (`magic`, a runtime register so that the mask stays an immediate) gives
+// 2^23 + c*2^(2i) exactly; adding `neg` = (-2^23, -2^23) leaves
+// (c_first 2^(2i), c_second 2^(2i)).  One logic op per code; the power of two
+// is folded into the multipliers (q' for keys, p' and a per-channel-pair
+// factor for values).
+__device__ __forceinline__ float2 code_pair(uint32_t w, uint32_t w16, int i, uint32_t magic,
+                                            float2 neg)
 {
-    const int p = i <= 10 ? 2 * i : 2 * i - 22;
-    const uint32_t src = i <= 10 ? w : w22;
-    return __uint_as_float((src & (3u << p)) | ((uint32_t)(150 - p) << 23));
+    const uint32_t msk = 3u << (2 * i);
+    uint32_t a, b;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(a) : "r"(w), "r"(msk), "r"(magic));
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(b) : "r"(w16), "r"(msk), "r"(magic));
+    return fadd2(make_float2(__uint_as_float(a), __uint_as_float(b)), neg);
 }
-__device__ __forceinline__ float code_magic(int i)
-{
-    const int p = i <= 10 ? 2 * i : 2 * i - 22;
-    return -__uint_as_float((uint32_t)(150 - p) << 23);
-}
-// Exact (c_i, c_{i+1}) as floats.
-__device__ __forceinline__ float2 code_pair(uint32_t w, uint32_t w22, int i)
-{
-    return fadd2(make_float2(code_raw(w, w22, i), code_raw(w, w22, i + 1)),
-                 make_float2(code_magic(i), code_magic(i + 1)));
-}
+// 2^-2i, the inverse of pair i's shift.
+__device__ __forceinline__ float pair_scale(int i) { return __uint_as_float((uint32_t)(127 - 2 * i) << 23); }
 
 template <int DT>
 __device__ __forceinline__ float to_f(uint16_t b)
@@ -153,11 +168,11 @@ template <int D, int HG, bool ROPE>
 struct WarpSmem {
     using L = Layout<D>;
     static constexpr int QPS = D / 4 + 4;           // padded q' slice (floats)
-    static constexpr int PPS = 36;                  // padded p' row (floats)
+    static constexpr int PPS = 34;                  // padded p' row (float2)
     static constexpr int RING = 0;                  // kStages x GB
     static constexpr int QP = kStages * L::GB;      // float [HG][4][QPS]
-    static constexpr int PP = QP + HG * 4 * QPS * 4;          // float [HG][NJ][PPS]
-    static constexpr int QS = PP + HG * L::NJ * PPS * 4;      // float [HG][D]
+    static constexpr int PP = QP + HG * 4 * QPS * 4;          // float2 [HG][NJ][PPS]
+    static constexpr int QS = PP + HG * L::NJ * PPS * 8;      // float [HG][D]
     static constexpr int SZ = QS + HG * D * 4;                // float2 [4][D/4] (RoPE)
     static constexpr int BAR = SZ + (ROPE ? D * 8 : 0);       // uint64 [kStages]
     static constexpr int BYTES = (BAR + kStages * 8 + 15) / 16 * 16;
@@ -167,7 +182,7 @@ template <int D, int HG, bool ROPE>
 struct DecodeShape {
     static constexpr int PER_WARP = WarpSmem<D, HG, ROPE>::BYTES;
     static constexpr int MAXW = 232448 / PER_WARP;
-    static constexpr int NW = MAXW > 16 ? 16 : MAXW;
+    static constexpr int NW = MAXW > KIVI_DECODE_MAXW ? KIVI_DECODE_MAXW : MAXW;
     static constexpr int SMEM = NW * PER_WARP;
 };
 
@@ -179,7 +194,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     using L = Layout<D>;
     using W = WarpSmem<D, HG, ROPE>;
     constexpr int NW = DecodeShape<D, HG, ROPE>::NW;
-    constexpr int CPL = L::CPL, NJ = L::NJ, KW = L::KW, HALF = L::HALF;
+    constexpr int CPL = L::CPL, QPL = L::QPL, NJ = L::NJ, KW = L::KW, HALF = L::HALF, TPW = L::TPW;
     constexpr int PSTRIDE = D + 4;
 
     extern __shared__ __align__(128) unsigned char smem_all[];
@@ -190,10 +205,12 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     unsigned char *ws = smem_all + warp * W::BYTES;
     unsigned char *ring = ws + W::RING;
     float *qp = (float *)(ws + W::QP);
-    float *pp = (float *)(ws + W::PP);
+    float2 *pp = (float2 *)(ws + W::PP);
     float *qs = (float *)(ws + W::QS);
     float2 *sz = (float2 *)(ws + W::SZ);
     const uint32_t bar0 = smem_addr(ws + W::BAR);
+    const uint32_t magic = p.magic;
+    const float2 neg = make_float2(p.neg_magic, p.neg_magic);
 
     Split sp;
     sp.init(p.seqs, p.n_groups, p.r, p.wg, p.wr, p.warps);
@@ -216,11 +233,15 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         }
     };
     pf_advance();
-    long long issued = 0, consumed = 0;
+    // Ring bookkeeping: items issued/consumed, the stage of the next issue,
+    // and the stage and phase parity of the next item to consume.
+    int issued = 0, consumed = 0, ist = 0, cst = 0;
+    uint32_t cph = 0;
     auto issue_next = [&]() {
         pf_advance();
         if (pf_i >= pf_e) return;
-        const int st = (int)(issued % kStages);
+        const int st = ist;
+        ist = ist + 1 == kStages ? 0 : ist + 1;
         if (lane == 0) {
             const uint32_t bar = bar0 + 8 * st;
             const uint32_t dst = smem_addr(ring + st * L::GB);
@@ -244,18 +265,27 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     for (int i = 0; i < kStages; ++i) issue_next();
 
     bool failed = false;
-    auto wait_stage = [&](long long k) -> bool {
-        const uint32_t bar = bar0 + 8 * (int)(k % kStages);
-        const uint32_t par = (uint32_t)((k / kStages) & 1);
+    auto wait_stage = [&]() -> bool {
+        const uint32_t bar = bar0 + 8 * cst;
         for (long long it = 0; it < kWaitLimit; ++it)
-            if (__all_sync(FULL, mbar_try_wait(bar, par))) return true;
+            if (__all_sync(FULL, mbar_try_wait(bar, cph))) return true;
         return false;
+    };
+    auto next_stage = [&]() {
+        ++consumed;
+        if (++cst == kStages) {
+            cst = 0;
+            cph ^= 1u;
+        }
     };
 
     const int tq = lane >> 2, cs = lane & 3;   // K mapping: 4 tokens x slice cs
     const int pcs = lane >> 3;                  // q' writer: permuted slice
-    const int pL0 = (lane & 7) * CPL;           //   and first local index
-    const int jl = lane * CPL / 32;             // V mapping: value group of lane
+    const int pL0 = (lane & 7) * QPL;           //   and first local index
+    const int vco = lane & 15, vth = lane >> 4; // V mapping: channel octet, token half
+    const int jl = vco * CPL / 32;              //   value group of the lane's channels
+    // V: token factor 2^(-CPL*(t mod TPW)) of token t = lane.
+    const float vtok = __uint_as_float((uint32_t)(127 - CPL * (lane % TPW)) << 23);
 
     for (long long s = s_first; s <= s_last && !failed; ++s) {
         long long i0, i1;
@@ -268,11 +298,14 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         __syncwarp();
         for (int i = lane; i < HG * D; i += 32) qs[i] = to_f<DT>(qg[i]) * p.qscale;
         __syncwarp();
-        float qreg[HG][CPL];
+        float qreg[HG][QPL], qsc[HG][QPL];
 #pragma unroll
         for (int h = 0; h < HG; ++h)
 #pragma unroll
-            for (int e = 0; e < CPL; ++e) qreg[h][e] = qs[h * D + k_channel<D>(pcs, pL0 + e)];
+            for (int e = 0; e < QPL; ++e) {
+                qreg[h][e] = qs[h * D + k_channel<D>(pcs, pL0 + e)];
+                qsc[h][e] = qreg[h][e] * pair_scale(((pL0 + e) & 15) >> 1);
+            }
 
         float m[HG], lsum[HG], zacc[HG][NJ];
         float2 accV[HG][CPL / 2];
@@ -287,7 +320,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         }
 
         // Online softmax update with the lane's score s_h for one token (or
-        // -inf), valid for the lane when `own` holds.
+        // -inf), counted in l when `own` holds.
         auto softmax_step = [&](float (&sc)[HG], float (&pr)[HG], bool own) {
 #pragma unroll
             for (int h = 0; h < HG; ++h) {
@@ -311,34 +344,42 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         };
 
         for (long long it = i0; it < i1; ++it) {
-            if (!wait_stage(consumed)) {
+            if (!wait_stage()) {
                 failed = true;
                 break;
             }
-            const unsigned char *st = ring + (int)(consumed % kStages) * L::GB;
+            const unsigned char *st = ring + cst * L::GB;
             if (it < p.n_groups) {
                 // ---------------- quantized group of 32 tokens ----------------
                 const uint16_t *km = (const uint16_t *)(st + L::KM + lane * (D / 8));
                 float bias[HG];
                 if constexpr (!ROPE) {
+                    float sk[QPL], zk[QPL];
+#pragma unroll
+                    for (int e = 0; e < QPL; ++e) {
+                        sk[e] = f16f(km[e]);
+                        zk[e] = f16f(km[QPL + e]);
+                    }
 #pragma unroll
                     for (int h = 0; h < HG; ++h) {
                         float bp = 0.f;
-                        float qv[CPL];
+                        float qv[QPL];
 #pragma unroll
-                        for (int e = 0; e < CPL; ++e) {
-                            qv[e] = qreg[h][e] * f16f(km[e]);
-                            bp = fmaf(qreg[h][e], f16f(km[CPL + e]), bp);
+                        for (int e = 0; e < QPL; ++e) {
+                            qv[e] = qsc[h][e] * sk[e];
+                            bp = fmaf(qreg[h][e], zk[e], bp);
                         }
                         float *dstq = qp + (h * 4 + pcs) * W::QPS + pL0;
 #pragma unroll
-                        for (int e = 0; e < CPL; e += 2) *(float2 *)(dstq + e) = make_float2(qv[e], qv[e + 1]);
+                        for (int e = 0; e < QPL; e += 2) *(float2 *)(dstq + e) = make_float2(qv[e], qv[e + 1]);
                         bias[h] = warp_sum(bp);
                     }
                 } else {
+                    // Scales carry the inverse of each code pair's shift.
 #pragma unroll
-                    for (int e = 0; e < CPL; ++e)
-                        sz[pcs * (D / 4) + pL0 + e] = make_float2(f16f(km[e]), f16f(km[CPL + e]));
+                    for (int e = 0; e < QPL; ++e)
+                        sz[pcs * (D / 4) + pL0 + e] =
+                            make_float2(f16f(km[e]) * pair_scale(((pL0 + e) & 15) >> 1), f16f(km[QPL + e]));
                 }
                 __syncwarp();
 
@@ -361,6 +402,9 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                         for (int h = 0; h < HG; ++h) acc[t][h] = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int k = 0; k < KW; ++k) {
+                        uint32_t kw16[4];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) kw16[t] = kw[t * KW + k] >> 16;
 #pragma unroll
                         for (int i = 0; i < 16; i += 4) {
                             float4 q4[HG];
@@ -369,9 +413,9 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                                 q4[h] = *(const float4 *)(qp + (h * 4 + cs) * W::QPS + 16 * k + i);
 #pragma unroll
                             for (int t = 0; t < 4; ++t) {
-                                const uint32_t w = kw[t * KW + k], w22 = w >> 22;
-                                const float2 c01 = code_pair(w, w22, i);
-                                const float2 c23 = code_pair(w, w22, i + 2);
+                                const uint32_t w = kw[t * KW + k];
+                                const float2 c01 = code_pair(w, kw16[t], i / 2, magic, neg);
+                                const float2 c23 = code_pair(w, kw16[t], i / 2 + 1, magic, neg);
 #pragma unroll
                                 for (int h = 0; h < HG; ++h) {
                                     acc[t][h] = ffma2(make_float2(q4[h].x, q4[h].y), c01, acc[t][h]);
@@ -392,10 +436,10 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                         float kh[D / 4];
 #pragma unroll
                         for (int k = 0; k < KW; ++k) {
-                            const uint32_t w = kw[t * KW + k], w22 = w >> 22;
+                            const uint32_t w = kw[t * KW + k], w16 = w >> 16;
 #pragma unroll
                             for (int i = 0; i < 16; i += 2) {
-                                const float2 c = code_pair(w, w22, i);
+                                const float2 c = code_pair(w, w16, i / 2, magic, neg);
                                 const float2 s0 = sz[cs * (D / 4) + 16 * k + i];
                                 const float2 s1 = sz[cs * (D / 4) + 16 * k + i + 1];
                                 kh[16 * k + i] = fmaf(c.x, s0.x, s0.y);
@@ -436,25 +480,29 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     float k1 = (hiB ? part[3][h] : part[1][h]) + __shfl_xor_sync(FULL, send1, 2);
                     float send = loB ? k0 : k1;
                     float keep = (loB ? k1 : k0) + __shfl_xor_sync(FULL, send, 1);
-                    sc[h] = ROPE ? keep : keep + bias[h];
+                    if constexpr (ROPE) sc[h] = keep;
+                    else sc[h] = keep + bias[h];
                 }
                 float pr[HG];
                 softmax_step(sc, pr, true);
 
-                // Value scales for token `lane`.
+                // Value scales for token `lane`; p' carries the token's
+                // power-of-two factor of the fast code path.
                 const uint16_t *vm = (const uint16_t *)(st + L::VM + lane * (D / 8));
 #pragma unroll
                 for (int j = 0; j < NJ; ++j) {
-                    const float svj = f16f(vm[j]), zvj = f16f(vm[NJ + j]);
+                    const float svj = f16f(vm[j]) * vtok, zvj = f16f(vm[NJ + j]);
 #pragma unroll
                     for (int h = 0; h < HG; ++h) {
-                        pp[(h * NJ + j) * W::PPS + lane] = pr[h] * svj;
+                        const float pv = pr[h] * svj;
+                        pp[(h * NJ + j) * W::PPS + lane] = make_float2(pv, pv);
                         zacc[h][j] = fmaf(pr[h], zvj, zacc[h][j]);
                     }
                 }
                 __syncwarp();
 
-                // Values: lane owns channels [lane*CPL, (lane+1)*CPL).
+                // Values: lane (vco, vth) owns channels [vco*CPL, (vco+1)*CPL)
+                // of tokens 16*vth .. 16*vth + 15.
                 uint32_t vw[L::WPL];
 #pragma unroll
                 for (int c = 0; c < L::WPL / 4; ++c) {
@@ -466,22 +514,23 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 }
 #pragma unroll
                 for (int u = 0; u < L::WPL; ++u) {
-                    const uint32_t w = vw[u], w22 = w >> 22;
+                    const uint32_t w = vw[u], w16 = w >> 16;
 #pragma unroll
-                    for (int t4 = 0; t4 < L::TPW; t4 += 4) {
+                    for (int t2 = 0; t2 < TPW; t2 += 2) {
                         float4 p4[HG];
 #pragma unroll
                         for (int h = 0; h < HG; ++h)
-                            p4[h] = *(const float4 *)(pp + (h * NJ + jl) * W::PPS + u * L::TPW + t4);
+                            p4[h] = *(const float4 *)(pp + (h * NJ + jl) * W::PPS + 16 * vth + u * TPW + t2);
 #pragma unroll
-                        for (int tt = 0; tt < 4; ++tt) {
+                        for (int tt = 0; tt < 2; ++tt) {
 #pragma unroll
-                            for (int c = 0; c < CPL; c += 2) {
-                                const float2 cc = code_pair(w, w22, (t4 + tt) * CPL + c);
+                            for (int mm = 0; mm < CPL / 2; ++mm) {
+                                const float2 cc = code_pair(w, w16, (t2 + tt) * (CPL / 2) + mm, magic, neg);
 #pragma unroll
                                 for (int h = 0; h < HG; ++h) {
-                                    const float pv = tt == 0 ? p4[h].x : tt == 1 ? p4[h].y : tt == 2 ? p4[h].z : p4[h].w;
-                                    accV[h][c / 2] = ffma2(make_float2(pv, pv), cc, accV[h][c / 2]);
+                                    const float2 pv = tt == 0 ? make_float2(p4[h].x, p4[h].y)
+                                                              : make_float2(p4[h].z, p4[h].w);
+                                    accV[h][mm] = ffma2(pv, cc, accV[h][mm]);
                                 }
                             }
                         }
@@ -543,14 +592,23 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 }
                 float pr[HG];
                 softmax_step(sc, pr, valid && cs == 0);
-                for (int t = 0; t < nt; ++t) {
-                    const uint16_t *vrow = rv + t * D + lane * CPL;
+                // Residual values: lane (vco, vth) takes tokens of parity vth,
+                // with the same per-pair factor 2^(2m) as the quantized codes.
+                for (int t0 = 0; t0 < nt; t0 += 2) {
+                    const int t = t0 + vth;
+                    const bool ok = t < nt;
                     float vx[CPL];
+                    if (ok) {
+                        const uint16_t *vrow = rv + t * D + vco * CPL;
 #pragma unroll
-                    for (int c = 0; c < CPL; ++c) vx[c] = to_f<DT>(vrow[c]);
+                        for (int c = 0; c < CPL; ++c) vx[c] = to_f<DT>(vrow[c]) * (float)(1 << (2 * (c / 2)));
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < CPL; ++c) vx[c] = 0.f;
+                    }
 #pragma unroll
                     for (int h = 0; h < HG; ++h) {
-                        const float pt = __shfl_sync(FULL, pr[h], 4 * t);
+                        const float pt = __shfl_sync(FULL, pr[h], 4 * (ok ? t : t0));
 #pragma unroll
                         for (int c = 0; c < CPL; c += 2)
                             accV[h][c / 2] = ffma2(make_float2(pt, pt), make_float2(vx[c], vx[c + 1]),
@@ -560,7 +618,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
             }
             // Stage consumed: refill it with the item kStages ahead.
             __syncwarp();
-            ++consumed;
+            next_stage();
             issue_next();
         }
         if (failed) break;
@@ -577,16 +635,30 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
 #pragma unroll
             for (int j = 0; j < NJ; ++j) zt[h][j] = warp_sum(zacc[h][j]);
         }
+        // Undo the per-pair factor 2^(2m), join the two token halves and add
+        // the zero term: lane (vco, vth) then holds channels vco*CPL + c.
+        float o[HG][CPL];
+#pragma unroll
+        for (int h = 0; h < HG; ++h)
+#pragma unroll
+            for (int c = 0; c < CPL; c += 2) {
+                const float2 a = accV[h][c / 2];
+                const float f = 1.0f / (float)(1 << (2 * (c / 2)));
+                const float x = a.x + __shfl_xor_sync(FULL, a.x, 16);
+                const float y = a.y + __shfl_xor_sync(FULL, a.y, 16);
+                o[h][c] = fmaf(x, f, zt[h][jl]);
+                o[h][c + 1] = fmaf(y, f, zt[h][jl]);
+            }
         float *outrow = p.out + (b * p.H_q + (long long)hk * HG) * D;
         if (count == 1) {
+            if (vth == 0) {
 #pragma unroll
-            for (int h = 0; h < HG; ++h) {
-                const float inv = 1.0f / lt[h];
+                for (int h = 0; h < HG; ++h) {
+                    const float inv = 1.0f / lt[h];
 #pragma unroll
-                for (int c = 0; c < CPL; c += 2) {
-                    const float2 o = accV[h][c / 2];
-                    *(float2 *)(outrow + h * D + lane * CPL + c) =
-                        make_float2((o.x + zt[h][jl]) * inv, (o.y + zt[h][jl]) * inv);
+                    for (int c = 0; c < CPL; c += 2)
+                        *(float2 *)(outrow + h * D + vco * CPL + c) =
+                            make_float2(o[h][c] * inv, o[h][c + 1] * inv);
                 }
             }
             continue;
@@ -594,13 +666,13 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         float *pbase = p.partials + ((s * p.slots) * HG) * (long long)PSTRIDE;
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
-            float *pr = pbase + ((long long)slot * HG + h) * PSTRIDE;
+            float *prow = pbase + ((long long)slot * HG + h) * PSTRIDE;
+            if (vth == 0) {
 #pragma unroll
-            for (int c = 0; c < CPL; c += 2) {
-                const float2 o = accV[h][c / 2];
-                *(float2 *)(pr + lane * CPL + c) = make_float2(o.x + zt[h][jl], o.y + zt[h][jl]);
+                for (int c = 0; c < CPL; c += 2)
+                    *(float2 *)(prow + vco * CPL + c) = make_float2(o[h][c], o[h][c + 1]);
             }
-            if (lane == 0) *(float2 *)(pr + D) = make_float2(m[h], lt[h]);
+            if (lane == 0) *(float2 *)(prow + D) = make_float2(m[h], lt[h]);
         }
         __syncwarp();
         int is_last = 0;
@@ -619,9 +691,9 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 mx = fmaxf(mx, __ldcg(pbase + ((long long)k * HG + h) * PSTRIDE + D));
             mx = warp_max(mx);
             float lacc = 0.f;
-            float o[CPL];
+            float oo[QPL];
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) o[c] = 0.f;
+            for (int c = 0; c < QPL; ++c) oo[c] = 0.f;
 #pragma unroll 4
             for (int k = 0; k < count; ++k) {
                 const float *pk = pbase + ((long long)k * HG + h) * PSTRIDE;
@@ -629,16 +701,16 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 const float wgt = ex2(ml.x - mx);
                 lacc = fmaf(wgt, ml.y, lacc);
 #pragma unroll
-                for (int c = 0; c < CPL; c += 2) {
-                    const float2 v = __ldcg((const float2 *)(pk + lane * CPL + c));
-                    o[c] = fmaf(wgt, v.x, o[c]);
-                    o[c + 1] = fmaf(wgt, v.y, o[c + 1]);
+                for (int c = 0; c < QPL; c += 2) {
+                    const float2 v = __ldcg((const float2 *)(pk + lane * QPL + c));
+                    oo[c] = fmaf(wgt, v.x, oo[c]);
+                    oo[c + 1] = fmaf(wgt, v.y, oo[c + 1]);
                 }
             }
             const float inv = 1.0f / lacc;
 #pragma unroll
-            for (int c = 0; c < CPL; c += 2)
-                *(float2 *)(outrow + h * D + lane * CPL + c) = make_float2(o[c] * inv, o[c + 1] * inv);
+            for (int c = 0; c < QPL; c += 2)
+                *(float2 *)(outrow + h * D + lane * QPL + c) = make_float2(oo[c] * inv, oo[c + 1] * inv);
         }
         if (lane == 0) p.tickets[s] = 0;
     }
@@ -647,8 +719,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         if (lane == 0) atomicCAS(p.err, 0, kErrWaitTimeout);
         // Let the copies already in flight land before the warp leaves.
         while (consumed < issued) {
-            wait_stage(consumed);
-            ++consumed;
+            wait_stage();
+            next_stage();
         }
     }
 }

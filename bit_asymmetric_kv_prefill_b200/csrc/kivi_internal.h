@@ -44,6 +44,8 @@ struct DecodeParams {
     long long warps;     // total warps of the split (<= total weight)
     int slots;           // partial slots per sequence
     float qscale;        // log2(e) / sqrt(D)
+    uint32_t magic;      // bits of 2^23 (the code-to-float exponent)
+    float neg_magic;     // -2^23
     const float *inv_freq;  // RoPE inverse frequencies [D/2] (pre-RoPE caches)
 };
 

@@ -7,11 +7,18 @@
 // group tile (32 tokens x D channels of K and of V) at a time:
 //   1. the tile is staged into padded shared memory with cp.async, double
 //      buffered across the CTA's groups;
-//   2. per-channel key min/max (one thread per channel) and per-token value
-//      min/max (warp-shuffle reductions over the 32 channels of a group) give
-//      the fp16 scale/zero and three exact fp32 code thresholds per group;
-//   3. every 32-bit word of 16 codes is built by one thread and the finished
-//      24*D-byte group block is written out with coalesced 16-byte stores.
+//   2. statistics: per-channel key min/max with paired (bf16x2 / f16x2)
+//      min/max over 16 rows per thread, the two row halves merged by a warp
+//      shuffle; per-token value min/max over each 32-channel group;
+//   3. each group's fp16 scale/zero and its three code thresholds.  The code
+//      clamp(rint(fl(x - z) / s), 0, 3) equals the number of thresholds x has
+//      reached, x_k being the smallest input value whose fp32 difference to z
+//      passes the k-th exact fp32 bound (see code_params); x_k is found by a
+//      bounded search around z + E_k that evaluates the definition itself;
+//   4. codes: two channels at a time, three paired `x >= x_k` compares give
+//      lane masks, two logic ops turn them into the pair's two 2-bit codes and
+//      one multiply-add shifts them into the word;
+//   5. the finished 24*D-byte group block leaves with coalesced 16-byte stores.
 // The residual rows of a prefill and the appended token of a flush are copied
 // by the same launch.
 #include <cuda_runtime.h>
@@ -21,11 +28,104 @@
 
 namespace kivi {
 
+// ---- input dtype helpers (bits are carried as uint16 / packed uint32) ----------
 template <int DT>
-__device__ __forceinline__ float to_f(uint16_t b)
+struct In;
+
+template <>
+struct In<1> {  // bfloat16
+    static constexpr uint16_t kInf = 0x7F80u, kNegInf = 0xFF80u;
+    __device__ static float f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+    __device__ static uint16_t from_double(double y) { return __bfloat16_as_ushort(__double2bfloat16(y)); }
+    __device__ static __nv_bfloat162 v(uint32_t u)
+    {
+        return __halves2bfloat162(__ushort_as_bfloat16((uint16_t)u), __ushort_as_bfloat16((uint16_t)(u >> 16)));
+    }
+    __device__ static uint32_t u(__nv_bfloat162 x)
+    {
+        return (uint32_t)__bfloat16_as_ushort(__low2bfloat16(x)) |
+               ((uint32_t)__bfloat16_as_ushort(__high2bfloat16(x)) << 16);
+    }
+    __device__ static uint32_t vmin(uint32_t a, uint32_t b) { return u(__hmin2(v(a), v(b))); }
+    __device__ static uint32_t vmax(uint32_t a, uint32_t b) { return u(__hmax2(v(a), v(b))); }
+    __device__ static uint32_t ge_mask(uint32_t a, uint32_t b) { return __hge2_mask(v(a), v(b)); }
+};
+
+template <>
+struct In<0> {  // IEEE fp16
+    static constexpr uint16_t kInf = 0x7C00u, kNegInf = 0xFC00u;
+    __device__ static float f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
+    __device__ static uint16_t from_double(double y) { return __half_as_ushort(__double2half(y)); }
+    __device__ static __half2 v(uint32_t u)
+    {
+        return __halves2half2(__ushort_as_half((uint16_t)u), __ushort_as_half((uint16_t)(u >> 16)));
+    }
+    __device__ static uint32_t u(__half2 x)
+    {
+        return (uint32_t)__half_as_ushort(__low2half(x)) | ((uint32_t)__half_as_ushort(__high2half(x)) << 16);
+    }
+    __device__ static uint32_t vmin(uint32_t a, uint32_t b) { return u(__hmin2(v(a), v(b))); }
+    __device__ static uint32_t vmax(uint32_t a, uint32_t b) { return u(__hmax2(v(a), v(b))); }
+    __device__ static uint32_t ge_mask(uint32_t a, uint32_t b) { return __hge2_mask(v(a), v(b)); }
+};
+
+// Neighbours in value order of a 16-bit sign-magnitude float (both zeros are
+// the value 0; the infinities are fixed points).
+template <int DT>
+__device__ __forceinline__ uint16_t next_up(uint16_t b)
 {
-    if constexpr (DT == 1) return __uint_as_float((uint32_t)b << 16);  // bf16
-    else return __half2float(__ushort_as_half(b));                     // fp16
+    if ((b & 0x7fffu) == 0) return 0x0001u;
+    if (b & 0x8000u) return (uint16_t)(b - 1);
+    return b == In<DT>::kInf ? b : (uint16_t)(b + 1);
+}
+template <int DT>
+__device__ __forceinline__ uint16_t next_down(uint16_t b)
+{
+    if ((b & 0x7fffu) == 0) return 0x8001u;
+    if (b & 0x8000u) return b == In<DT>::kNegInf ? b : (uint16_t)(b + 1);
+    return (uint16_t)(b - 1);
+}
+
+// Does input value x reach threshold e: fl32(x - z) > e (the definition's
+// fp32 subtraction, compared against the exact fp32 bound)?
+template <int DT>
+__device__ __forceinline__ bool passes(uint16_t x, float e, float z)
+{
+    return __fsub_rn(In<DT>::f(x), z) > e;
+}
+
+// Smallest input value x (as bits) with fl32(x - z) > e; +inf when none.
+// fl32(x - z) is non-decreasing in x, so {x : passes} is an upper set; the
+// start point rounds z + e to the input dtype and a few bounded steps settle
+// on its least element.
+template <int DT>
+__device__ __forceinline__ uint16_t min_passing(float e, float z)
+{
+    if (!(e < __int_as_float(0x7f800000))) return In<DT>::kInf;
+    uint16_t x = In<DT>::from_double((double)e + (double)z);
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {
+        const uint16_t d = next_down<DT>(x);
+        if (d == x || !passes<DT>(d, e, z)) break;
+        x = d;
+    }
+#pragma unroll 1
+    for (int i = 0; i < 8 && !passes<DT>(x, e, z); ++i) x = next_up<DT>(x);
+    return x;
+}
+
+// Two codes of a channel pair x (packed) against packed thresholds t1..t3:
+// bit pattern (c_lo at bits 0-1, c_hi at bits 16-17).  Masks m_k are 0xffff
+// per half where x >= t_k; since m1 >= m2 >= m3, bit1 of a code is m2 and
+// bit0 is m1 ^ m2 ^ m3.
+template <int DT>
+__device__ __forceinline__ uint32_t code_pair_bits(uint32_t x, uint32_t t1, uint32_t t2, uint32_t t3)
+{
+    const uint32_t m1 = In<DT>::ge_mask(x, t1), m2 = In<DT>::ge_mask(x, t2), m3 = In<DT>::ge_mask(x, t3);
+    uint32_t a, r;
+    asm("lop3.b32 %0, %1, %2, %3, 0x28;" : "=r"(a) : "r"(m1), "r"(m3), "r"(0x00010001u));  // (m1^m3)&K
+    asm("lop3.b32 %0, %1, %2, %3, 0x78;" : "=r"(r) : "r"(a), "r"(m2), "r"(0x00030003u));  // a^(m2&M)
+    return r;
 }
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
@@ -37,19 +137,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__device__ __forceinline__ float warp_min(float x)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
-    return x;
-}
-__device__ __forceinline__ float warp_max(float x)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-    return x;
-}
-
 constexpr int kQuantThreads = 256;
 
 template <int D>
@@ -57,109 +144,119 @@ struct QuantSmem {
     static constexpr int RS = D + 8;                      // padded row, elements
     static constexpr int TILE = 32 * RS;                  // one K or V tile
     static constexpr int TILES_BYTES = 2 * 2 * TILE * 2;  // 2 buffers x (K, V)
-    static constexpr int STATK = TILES_BYTES;             // float4 [D]
-    static constexpr int STATV = STATK + D * 16;          // float4 [32][D/32]
-    static constexpr int OUTB = STATV + 32 * (D / 32) * 16;
+    static constexpr int THRK = TILES_BYTES;              // uint16 [3][D]
+    static constexpr int THRV = THRK + 3 * D * 2;         // uint16 [32][D/32][4]
+    static constexpr int OUTB = (THRV + 32 * (D / 32) * 8 + 15) / 16 * 16;
     static constexpr int BYTES = OUTB + 24 * D;
 };
 
 template <int D, int DT>
 __device__ void quantize_tile(const QuantParams &p, long long item, const uint16_t *tk,
-                              const uint16_t *tv, float4 *statK, float4 *statV, uint8_t *outb)
+                              const uint16_t *tv, uint16_t *thrK, uint16_t *thrV, uint8_t *outb)
 {
     using L = Layout<D>;
+    using H = In<DT>;
     constexpr int RS = QuantSmem<D>::RS;
+    constexpr int NJ = L::NJ, CPL = L::CPL, TPW = L::TPW, KW = L::KW;
     const int tid = threadIdx.x;
     const long long s = item / p.n_g;
     const int g = (int)(item % p.n_g);
 
     if (tid < D) {
-        // Keys, per channel: min/max over the 32 tokens of channel tid.
-        float mn = to_f<DT>(tk[tid]), mx = mn;
-#pragma unroll 8
-        for (int t = 1; t < 32; ++t) {
-            float x = to_f<DT>(tk[t * RS + tid]);
-            mn = fminf(mn, x);
-            mx = fmaxf(mx, x);
-        }
-        CodeParams cp = code_params(mn, mx);
-        statK[tid] = make_float4(cp.e1, cp.e2, cp.e3, cp.z);
-        int off = L::KM + km_offset<D>(k_perm_index<D>(tid));
-        *(uint16_t *)(outb + off) = cp.s_bits;
-        *(uint16_t *)(outb + off + D / 16) = cp.z_bits;
-    } else {
-        // Values, per token: warp-shuffle min/max over 32 channels.
-        const int nvw = (kQuantThreads - D) / 32;
-        const int w = (tid - D) >> 5, lane = tid & 31;
-        for (int t = w; t < 32; t += nvw) {
+        // Keys, per channel: thread (pair cp, row half hh) takes 16 rows of a
+        // channel pair; the halves meet through a shuffle with lane ^ 1.
+        const int cp = tid >> 1, hh = tid & 1;
+        const uint16_t *col = tk + hh * 16 * RS + 2 * cp;
+        uint32_t mn = *(const uint32_t *)col, mx = mn;
 #pragma unroll
-            for (int j = 0; j < L::NJ; ++j) {
-                float x = to_f<DT>(tv[t * RS + j * 32 + lane]);
-                float mn = warp_min(x), mx = warp_max(x);
-                if (lane == 0) {
-                    CodeParams cp = code_params(mn, mx);
-                    statV[t * L::NJ + j] = make_float4(cp.e1, cp.e2, cp.e3, cp.z);
-                    int off = L::VM + t * (D / 8) + j * 2;
-                    *(uint16_t *)(outb + off) = cp.s_bits;
-                    *(uint16_t *)(outb + off + D / 16) = cp.z_bits;
-                }
+        for (int r = 1; r < 16; ++r) {
+            const uint32_t v = *(const uint32_t *)(col + r * RS);
+            mn = H::vmin(mn, v);
+            mx = H::vmax(mx, v);
+        }
+        mn = H::vmin(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+        mx = H::vmax(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        const int ch = 2 * cp + hh;
+        const uint16_t mnb = (uint16_t)(hh ? mn >> 16 : mn), mxb = (uint16_t)(hh ? mx >> 16 : mx);
+        const CodeParams c = code_params(H::f(mnb), H::f(mxb));
+        thrK[ch] = min_passing<DT>(c.e1, c.z);
+        thrK[D + ch] = min_passing<DT>(c.e2, c.z);
+        thrK[2 * D + ch] = min_passing<DT>(c.e3, c.z);
+        const int off = L::KM + km_offset<D>(k_perm_index<D>(ch));
+        *(uint16_t *)(outb + off) = c.s_bits;
+        *(uint16_t *)(outb + off + D / 16) = c.z_bits;
+    } else {
+        // Values, per token: one (token, 32-channel group) per thread.
+        for (int qd = tid - D; qd < 32 * NJ; qd += kQuantThreads - D) {
+            const int t = qd / NJ, j = qd % NJ;
+            const uint4 *row = (const uint4 *)(tv + t * RS + j * 32);
+            uint4 a = row[0];
+            uint32_t mn = H::vmin(a.x, a.y), mx = H::vmax(a.x, a.y);
+            mn = H::vmin(mn, H::vmin(a.z, a.w));
+            mx = H::vmax(mx, H::vmax(a.z, a.w));
+#pragma unroll
+            for (int q = 1; q < 4; ++q) {
+                a = row[q];
+                mn = H::vmin(mn, H::vmin(H::vmin(a.x, a.y), H::vmin(a.z, a.w)));
+                mx = H::vmax(mx, H::vmax(H::vmax(a.x, a.y), H::vmax(a.z, a.w)));
             }
+            mn = H::vmin(mn, (mn >> 16) | (mn << 16));
+            mx = H::vmax(mx, (mx >> 16) | (mx << 16));
+            const CodeParams c = code_params(H::f((uint16_t)mn), H::f((uint16_t)mx));
+            uint16_t *tr = thrV + (t * NJ + j) * 4;
+            tr[0] = min_passing<DT>(c.e1, c.z);
+            tr[1] = min_passing<DT>(c.e2, c.z);
+            tr[2] = min_passing<DT>(c.e3, c.z);
+            const int off = L::VM + t * (D / 8) + j * 2;
+            *(uint16_t *)(outb + off) = c.s_bits;
+            *(uint16_t *)(outb + off + D / 16) = c.z_bits;
         }
     }
     __syncthreads();
 
-    // Key code words: thread -> (lane, token pair, word slot k); tokens tok and
-    // tok+2 of the lane share the 16 channels, so their thresholds load once.
     if (tid < D) {
-        const int lane = tid / (2 * L::KW), rem = tid % (2 * L::KW);
-        const int tokp = rem / L::KW, k = rem % L::KW;
+        // Key code words: thread -> (lane, token pair, word slot k); tokens tok
+        // and tok+2 of the lane share the word's 16 channels and thresholds.
+        const int lane = tid / (2 * KW), rem = tid % (2 * KW);
+        const int tokp = rem / KW, k = rem % KW;
         const int cs = lane & 3, tq = lane >> 2;
-        constexpr int RUN = (D / 8) < 16 ? (D / 8) : 16;  // contiguous channels
-        float4 th[16];
+        uint32_t t1[8], t2[8], t3[8];
+        int ch0[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) th[i] = statK[k_channel<D>(cs, 16 * k + i)];
+        for (int i = 0; i < 8; ++i) {
+            ch0[i] = k_channel<D>(cs, 16 * k + 2 * i);
+            t1[i] = *(const uint32_t *)(thrK + ch0[i]);
+            t2[i] = *(const uint32_t *)(thrK + D + ch0[i]);
+            t3[i] = *(const uint32_t *)(thrK + 2 * D + ch0[i]);
+        }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int tok = tokp + 2 * h;
-            const int t = 4 * tq + tok;
+            const uint16_t *row = tk + (4 * tq + tok) * RS;
             uint32_t word = 0;
 #pragma unroll
-            for (int r0 = 0; r0 < 16; r0 += RUN) {
-                const int c0 = k_channel<D>(cs, 16 * k + r0);
-                uint16_t xs[RUN];
-#pragma unroll
-                for (int v = 0; v < RUN; v += 8)
-                    *(uint4 *)&xs[v] = *(const uint4 *)&tk[t * RS + c0 + v];
-#pragma unroll
-                for (int i = 0; i < RUN; ++i) {
-                    const float4 e = th[r0 + i];
-                    word |= code_of(to_f<DT>(xs[i]), e.w, e.x, e.y, e.z) << (2 * (r0 + i));
-                }
-            }
-            *(uint32_t *)(outb + L::KC + code_word_offset(lane, tok * L::KW + k)) = word;
+            for (int i = 7; i >= 0; --i)
+                word = word * 4u + code_pair_bits<DT>(*(const uint32_t *)(row + ch0[i]), t1[i], t2[i], t3[i]);
+            *(uint32_t *)(outb + L::KC + code_word_offset(lane, tok * KW + k)) = word;
         }
-    }
-    // Value code words: thread -> (lane, word u); TPW tokens x CPL channels.
-    for (int vp = tid; vp < 2 * D; vp += kQuantThreads) {
-        const int lane = vp / L::WPL, u = vp % L::WPL;
-        const int j = lane * L::CPL / 32;
-        uint32_t word = 0;
+    } else {
+        // Value code words: thread -> (lane = 16*th + co, word u).
+        for (int vp = tid - D; vp < 2 * D; vp += kQuantThreads - D) {
+            const int lane = vp / L::WPL, u = vp % L::WPL;
+            const int co = lane & 15, th = lane >> 4;
+            const int j = co * CPL / 32;
+            uint32_t word = 0;
 #pragma unroll
-        for (int tt = 0; tt < L::TPW; ++tt) {
-            const int t = u * L::TPW + tt;
-            const float4 e = statV[t * L::NJ + j];
-            uint16_t xs[L::CPL];
-            if constexpr (L::CPL == 4) {
-                *(uint2 *)xs = *(const uint2 *)&tv[t * RS + lane * 4];
-            } else {
-#pragma unroll
-                for (int c = 0; c < L::CPL; ++c) xs[c] = tv[t * RS + lane * L::CPL + c];
+            for (int i = 7; i >= 0; --i) {
+                const int tt = i / (CPL / 2), m = i % (CPL / 2);
+                const int t = 16 * th + u * TPW + tt;
+                const uint16_t *tr = thrV + (t * NJ + j) * 4;
+                const uint32_t b1 = tr[0], b2 = tr[1], b3 = tr[2];
+                const uint32_t x = *(const uint32_t *)(tv + t * RS + co * CPL + 2 * m);
+                word = word * 4u + code_pair_bits<DT>(x, b1 | (b1 << 16), b2 | (b2 << 16), b3 | (b3 << 16));
             }
-#pragma unroll
-            for (int c = 0; c < L::CPL; ++c)
-                word |= code_of(to_f<DT>(xs[c]), e.w, e.x, e.y, e.z) << (2 * (tt * L::CPL + c));
+            *(uint32_t *)(outb + L::VC + code_word_offset(lane, u)) = word;
         }
-        *(uint32_t *)(outb + L::VC + code_word_offset(lane, u)) = word;
     }
     __syncthreads();
 
@@ -179,13 +276,13 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
 }
 
 template <int D, int DT>
-__global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantParams p)
+__global__ void __launch_bounds__(kQuantThreads, 3) quant_kernel(QuantParams p)
 {
     using S = QuantSmem<D>;
     extern __shared__ __align__(16) unsigned char smem[];
     uint16_t *tiles = (uint16_t *)smem;
-    float4 *statK = (float4 *)(smem + S::STATK);
-    float4 *statV = (float4 *)(smem + S::STATV);
+    uint16_t *thrK = (uint16_t *)(smem + S::THRK);
+    uint16_t *thrV = (uint16_t *)(smem + S::THRV);
     uint8_t *outb = smem + S::OUTB;
 
     const long long n_group_items = p.seqs * (long long)p.n_g;
@@ -219,7 +316,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantParams p)
         __syncthreads();
         if (item < n_group_items) {
             quantize_tile<D, DT>(p, item, tiles + (buf * 2 + 0) * S::TILE,
-                                 tiles + (buf * 2 + 1) * S::TILE, statK, statV, outb);
+                                 tiles + (buf * 2 + 1) * S::TILE, thrK, thrV, outb);
         } else {
             // Prefill residual: rows [copy_row0, copy_row0 + r_copy) -> slots.
             const long long s = item - n_group_items;
@@ -264,16 +361,18 @@ template <int D, int DT>
 static cudaError_t launch_quant_t(const QuantParams &p, cudaStream_t st)
 {
     using S = QuantSmem<D>;
-    static bool configured = false;
-    if (!configured) {
+    static int configured_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured_dev != dev) {
         cudaError_t e = cudaFuncSetAttribute(quant_kernel<D, DT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured_dev = dev;
     }
     const long long items = p.seqs * (long long)p.n_g + (p.r_copy > 0 ? p.seqs : 0);
     if (items == 0) return cudaSuccess;
-    long long grid = (long long)num_sms() * 4;
+    long long grid = (long long)num_sms() * 3;
     if (grid > items) grid = items;
     quant_kernel<D, DT><<<(unsigned)grid, kQuantThreads, S::BYTES, st>>>(p);
     return cudaGetLastError();

@@ -65,7 +65,6 @@ def lib():
     L.oracle_decode_seq.argtypes = [u16p, c_int, c_int, c_int, c_int, c_int, c_int, c_d,
                                     u8p, u16p, u16p, u8p, u16p, u16p, u16p, u16p, c_ll, c_int,
                                     f64p, f32p]
-    L.oracle_attention_raw.argtypes = [u16p, c_int, c_int, c_int, u16p, u16p, c_ll, f64p, f32p]
     L.oracle_rope_inv_freq.argtypes = [c_int, c_d, f32p]
     L.oracle_rope_row.argtypes = [f64p, c_int, c_ll, f32p]
     L.oracle_kv_bytes.argtypes = [c_ll, c_ll, c_ll, c_ll, c_ll, c_int, c_int, c_ll, f64p]
@@ -132,19 +131,6 @@ def kv_bytes(layers, heads, head_dim, R, context, bits=2, dtype_bytes=2, G=32):
     keys = ["grouped_per_token", "residual_total", "residual_per_token", "sum_per_token",
             "full_per_token", "reduction", "metadata_per_token"]
     return dict(zip(keys, out.tolist()))
-
-
-def attention_raw(q: np.ndarray, K: np.ndarray, V: np.ndarray, dtype: int) -> np.ndarray:
-    """Textbook softmax attention: q [HG, D], K/V [T, D] (uint16 bits)."""
-    q, K, V = (np.ascontiguousarray(a, dtype=np.uint16) for a in (q, K, V))
-    HG, D = q.shape
-    T = K.shape[0]
-    out = np.zeros((HG, D), np.float32)
-    sc = np.zeros(max(T, 1), np.float64)
-    lib().oracle_attention_raw(_ptr(q, ctypes.c_uint16), HG, D, dtype, _ptr(K, ctypes.c_uint16),
-                               _ptr(V, ctypes.c_uint16), T, _ptr(sc, ctypes.c_double),
-                               _ptr(out, ctypes.c_float))
-    return out
 
 
 # ---- the cache --------------------------------------------------------------

@@ -313,34 +313,6 @@ void oracle_decode_seq(const uint16_t *q, int HG, int D, int G, int R, int dtype
     }
 }
 
-/* Textbook attention on raw rows K, V [T][D] (no quantization), for pins. */
-void oracle_attention_raw(const uint16_t *q, int HG, int D, int dtype,
-                          const uint16_t *K, const uint16_t *V, long long T,
-                          double *scores, float *out)
-{
-    double inv_sqrt_d = 1.0 / sqrt((double)D);
-    for (int h = 0; h < HG; ++h) {
-        double m = -INFINITY;
-        for (long long t = 0; t < T; ++t) {
-            double s = 0.0;
-            for (int d = 0; d < D; ++d)
-                s += (double)load_elem(q, (long long)h * D + d, dtype) *
-                     (double)load_elem(K, t * D + d, dtype);
-            s *= inv_sqrt_d;
-            scores[t] = s;
-            if (s > m) m = s;
-        }
-        double l = 0.0;
-        for (long long t = 0; t < T; ++t) l += exp(scores[t] - m);
-        for (int d = 0; d < D; ++d) {
-            double a = 0.0;
-            for (long long t = 0; t < T; ++t)
-                a += exp(scores[t] - m) * (double)load_elem(V, t * D + d, dtype);
-            out[(long long)h * D + d] = (float)(a / l);
-        }
-    }
-}
-
 /* ---- byte accounting ----------------------------------------------------- */
 
 /*
