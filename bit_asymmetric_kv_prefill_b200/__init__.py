@@ -72,6 +72,7 @@ def lib():
     L.kivi_prefill.argtypes = [vp, vp, vp, i64, vp]
     L.kivi_append.argtypes = [vp, vp, vp, vp]
     L.kivi_decode_attn.argtypes = [vp, vp, i32, vp, vp]
+    L.kivi_decode_attn_noalloc.argtypes = [vp, vp, i32, vp, vp]
     L.kivi_cache_reset.argtypes = [vp]
     L.kivi_cache_length.argtypes = [vp, P(i64), P(i32)]
     L.kivi_cache_bytes.argtypes = [vp, P(_Bytes)]
@@ -80,7 +81,8 @@ def lib():
     L.kivi_cache_destroy.argtypes = [vp]
     L.kivi_decode_split.argtypes = [i64, i64, i32, i32, i32, i64, i64, i64, P(i64)]
     for name in ("kivi_cache_create", "kivi_cache_create_ex", "kivi_cache_required_bytes",
-                 "kivi_prefill", "kivi_append", "kivi_decode_attn", "kivi_cache_reset",
+                 "kivi_prefill", "kivi_append", "kivi_decode_attn", "kivi_decode_attn_noalloc",
+                 "kivi_cache_reset",
                  "kivi_cache_length", "kivi_cache_bytes", "kivi_export", "kivi_device_status",
                  "kivi_cache_destroy", "kivi_decode_split"):
         getattr(L, name).restype = st
@@ -195,6 +197,19 @@ class KiviCache:
             raise ValueError("out must be a contiguous CUDA float32 [B, H_q, D] tensor")
         _check(lib().kivi_decode_attn(self._h, qp, H_q, out.data_ptr(), _stream_ptr(stream)),
                "kivi_decode_attn")
+        return out
+
+    def decode_noalloc(self, q: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+        """Decode into a caller-provided `out` without any device allocation:
+        the library keeps this call's scratch in a fixed 8 MiB device array
+        (see kivi_decode_attn_noalloc), for hosts that may not allocate."""
+        H_q = q.shape[1]
+        qp = self._tensor(q, (self.B, H_q, self.D), "q")
+        if (out.dtype != torch.float32 or tuple(out.shape) != (self.B, H_q, self.D)
+                or not out.is_contiguous() or not out.is_cuda):
+            raise ValueError("out must be a contiguous CUDA float32 [B, H_q, D] tensor")
+        _check(lib().kivi_decode_attn_noalloc(self._h, qp, H_q, out.data_ptr(), _stream_ptr(stream)),
+               "kivi_decode_attn_noalloc")
         return out
 
     def reset(self):

@@ -501,3 +501,55 @@ extern "C" kivi_status kivi_decode_split(long long seqs, long long n_groups, int
     out[3] = i1;
     return KIVI_OK;
 }
+
+namespace kivi {
+
+// Launch parameters of a decode call on cache c, validated exactly as
+// kivi_decode_attn validates them, with the scratch pointers (partials,
+// tickets) and the partial slot count left for the caller to fill.
+kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q, float *out,
+                                           DecodeParams *p, int *D, int *HG, int *dtype,
+                                           int *pre_rope)
+{
+    if (!c || !q || !out || !p || !aligned16(q) || !aligned16(out)) return KIVI_ERR_ARG;
+    if (!c->prefilled) return KIVI_ERR_STATE;
+    if (H_q < 1 || H_q % c->cfg.H_kv != 0) return KIVI_ERR_ARG;
+    const int hg = H_q / c->cfg.H_kv;
+    const int nw = decode_warps_per_cta(c->cfg.D, hg, c->cfg.pre_rope);
+    if (nw == 0 || hg > kMaxGroupHeads) return KIVI_ERR_UNSUPPORTED;
+    Split sp;
+    sp.init(c->plan.seqs, c->n_q / kG, c->r, c->wg, c->wr, 1);
+    long long warps = (long long)c->sms * nw;
+    if (warps > sp.Tot) warps = sp.Tot;
+    p->packed = c->packed;
+    p->ngcap = c->plan.ngcap;
+    p->resK = c->resK;
+    p->resV = c->resV;
+    p->R = c->cfg.R;
+    p->q = (const uint16_t *)q;
+    p->out = out;
+    p->partials = nullptr;
+    p->tickets = nullptr;
+    p->err = c->err;
+    p->H_kv = c->cfg.H_kv;
+    p->H_q = H_q;
+    p->seqs = c->plan.seqs;
+    p->n_groups = c->n_q / kG;
+    p->r = c->r;
+    p->n_q = c->n_q;
+    p->wg = c->wg;
+    p->wr = c->wr;
+    p->warps = warps;
+    p->slots = (int)(warps / p->seqs + 2);
+    p->qscale = (float)(1.4426950408889634 / std::sqrt((double)c->cfg.D));
+    p->inv_freq = c->inv_freq;
+    p->magic = 0x4B000000u;
+    p->neg_magic = -8388608.0f;
+    *D = c->cfg.D;
+    *HG = hg;
+    *dtype = c->cfg.dtype;
+    *pre_rope = c->cfg.pre_rope;
+    return KIVI_OK;
+}
+
+}  // namespace kivi

@@ -134,6 +134,32 @@ KIVI_API kivi_status kivi_append(kivi_cache *c, const void *k_t, const void *v_t
 KIVI_API kivi_status kivi_decode_attn(kivi_cache *c, const void *q, int H_q, float *out,
                              void *stream);
 
+/*
+ * Decode attention exactly as kivi_decode_attn, for callers that must not
+ * allocate device memory (no part of the method corresponds to this call: it
+ * only changes where the decode's scratch lives).  Engines that plan all
+ * device memory ahead and forbid allocation while serving, plugins that only
+ * receive pointers from their host, and paths that cannot afford cudaMalloc's
+ * device-wide synchronisation can use it: the split-K partials and
+ * per-sequence tickets go into one fixed 8 MiB (8,388,608-byte) array inside
+ * the library, which every GPU that loads the library holds until the process
+ * exits.  The call itself
+ * allocates nothing and calls no allocating routine.
+ *   - The first call on a device looks up that array's device address (once
+ *     per device, with the device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the array and it keeps the last call's contents; the
+ *     call clears the tickets it needs on `stream` before its kernel.  Calls
+ *     whose kernels overlap on the GPU (any caches, any streams) race on the
+ *     array: order them, e.g. on one stream.
+ *   - Returns KIVI_ERR_CAPACITY, launching nothing, when the call's scratch
+ *     (tickets for B*H_kv sequences plus B*H_kv*slots*(H_q/H_kv)*(D+4) fp32
+ *     partials, slots = warps/(B*H_kv) + 2) exceeds the array.
+ * Arguments, layouts and other errors as kivi_decode_attn.
+ */
+KIVI_API kivi_status kivi_decode_attn_noalloc(kivi_cache *c, const void *q, int H_q, float *out,
+                                              void *stream);
+
 /* Forget the cached tokens (host counters only; device buffers are kept). */
 KIVI_API kivi_status kivi_cache_reset(kivi_cache *c);
 
