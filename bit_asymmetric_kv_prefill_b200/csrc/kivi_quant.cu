@@ -21,6 +21,8 @@
 //   5. the finished 24*D-byte group block leaves with coalesced 16-byte stores.
 // The residual rows of a prefill and the appended token of a flush are copied
 // by the same launch.
+#include <cstring>
+
 #include <cuda_runtime.h>
 
 #include "kivi_common.cuh"
@@ -39,12 +41,15 @@ struct In<1> {  // bfloat16
     __device__ static uint16_t from_double(double y) { return __bfloat16_as_ushort(__double2bfloat16(y)); }
     __device__ static __nv_bfloat162 v(uint32_t u)
     {
-        return __halves2bfloat162(__ushort_as_bfloat16((uint16_t)u), __ushort_as_bfloat16((uint16_t)(u >> 16)));
+        __nv_bfloat162 r;
+        memcpy(&r, &u, 4);
+        return r;
     }
     __device__ static uint32_t u(__nv_bfloat162 x)
     {
-        return (uint32_t)__bfloat16_as_ushort(__low2bfloat16(x)) |
-               ((uint32_t)__bfloat16_as_ushort(__high2bfloat16(x)) << 16);
+        uint32_t r;
+        memcpy(&r, &x, 4);
+        return r;
     }
     __device__ static uint32_t vmin(uint32_t a, uint32_t b) { return u(__hmin2(v(a), v(b))); }
     __device__ static uint32_t vmax(uint32_t a, uint32_t b) { return u(__hmax2(v(a), v(b))); }
@@ -58,11 +63,15 @@ struct In<0> {  // IEEE fp16
     __device__ static uint16_t from_double(double y) { return __half_as_ushort(__double2half(y)); }
     __device__ static __half2 v(uint32_t u)
     {
-        return __halves2half2(__ushort_as_half((uint16_t)u), __ushort_as_half((uint16_t)(u >> 16)));
+        __half2 r;
+        memcpy(&r, &u, 4);
+        return r;
     }
     __device__ static uint32_t u(__half2 x)
     {
-        return (uint32_t)__half_as_ushort(__low2half(x)) | ((uint32_t)__half_as_ushort(__high2half(x)) << 16);
+        uint32_t r;
+        memcpy(&r, &x, 4);
+        return r;
     }
     __device__ static uint32_t vmin(uint32_t a, uint32_t b) { return u(__hmin2(v(a), v(b))); }
     __device__ static uint32_t vmax(uint32_t a, uint32_t b) { return u(__hmax2(v(a), v(b))); }
@@ -168,12 +177,18 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
         const int cp = tid >> 1, hh = tid & 1;
         const uint16_t *col = tk + hh * 16 * RS + 2 * cp;
         uint32_t mn = *(const uint32_t *)col, mx = mn;
+        uint32_t mn1 = *(const uint32_t *)(col + RS), mx1 = mn1;
 #pragma unroll
-        for (int r = 1; r < 16; ++r) {
-            const uint32_t v = *(const uint32_t *)(col + r * RS);
-            mn = H::vmin(mn, v);
-            mx = H::vmax(mx, v);
+        for (int r = 2; r < 16; r += 2) {
+            const uint32_t v0 = *(const uint32_t *)(col + r * RS);
+            const uint32_t v1 = *(const uint32_t *)(col + (r + 1) * RS);
+            mn = H::vmin(mn, v0);
+            mx = H::vmax(mx, v0);
+            mn1 = H::vmin(mn1, v1);
+            mx1 = H::vmax(mx1, v1);
         }
+        mn = H::vmin(mn, mn1);
+        mx = H::vmax(mx, mx1);
         mn = H::vmin(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
         mx = H::vmax(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         const int ch = 2 * cp + hh;
@@ -220,23 +235,41 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
         const int lane = tid / (2 * KW), rem = tid % (2 * KW);
         const int tokp = rem / KW, k = rem % KW;
         const int cs = lane & 3, tq = lane >> 2;
+        // The word's 16 channels come in runs of RUN contiguous channels
+        // (one run when D >= 128, one per RoPE half when D == 64).
+        constexpr int RUN = L::HALF < 16 ? L::HALF : 16;
         uint32_t t1[8], t2[8], t3[8];
-        int ch0[8];
+        int base[16 / RUN];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            ch0[i] = k_channel<D>(cs, 16 * k + 2 * i);
-            t1[i] = *(const uint32_t *)(thrK + ch0[i]);
-            t2[i] = *(const uint32_t *)(thrK + D + ch0[i]);
-            t3[i] = *(const uint32_t *)(thrK + 2 * D + ch0[i]);
+        for (int r = 0; r < 16 / RUN; ++r) {
+            base[r] = k_channel<D>(cs, 16 * k + r * RUN);
+#pragma unroll
+            for (int v = 0; v < RUN / 8; ++v) {
+                const uint4 a = *(const uint4 *)(thrK + base[r] + 8 * v);
+                const uint4 b = *(const uint4 *)(thrK + D + base[r] + 8 * v);
+                const uint4 c = *(const uint4 *)(thrK + 2 * D + base[r] + 8 * v);
+                const int i0 = r * (RUN / 2) + 4 * v;
+                t1[i0] = a.x; t1[i0 + 1] = a.y; t1[i0 + 2] = a.z; t1[i0 + 3] = a.w;
+                t2[i0] = b.x; t2[i0 + 1] = b.y; t2[i0 + 2] = b.z; t2[i0 + 3] = b.w;
+                t3[i0] = c.x; t3[i0 + 1] = c.y; t3[i0 + 2] = c.z; t3[i0 + 3] = c.w;
+            }
         }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int tok = tokp + 2 * h;
             const uint16_t *row = tk + (4 * tq + tok) * RS;
+            uint32_t x[8];
+#pragma unroll
+            for (int r = 0; r < 16 / RUN; ++r)
+#pragma unroll
+                for (int v = 0; v < RUN / 8; ++v) {
+                    const uint4 a = *(const uint4 *)(row + base[r] + 8 * v);
+                    const int i0 = r * (RUN / 2) + 4 * v;
+                    x[i0] = a.x; x[i0 + 1] = a.y; x[i0 + 2] = a.z; x[i0 + 3] = a.w;
+                }
             uint32_t word = 0;
 #pragma unroll
-            for (int i = 7; i >= 0; --i)
-                word = word * 4u + code_pair_bits<DT>(*(const uint32_t *)(row + ch0[i]), t1[i], t2[i], t3[i]);
+            for (int i = 7; i >= 0; --i) word = word * 4u + code_pair_bits<DT>(x[i], t1[i], t2[i], t3[i]);
             *(uint32_t *)(outb + L::KC + code_word_offset(lane, tok * KW + k)) = word;
         }
     } else {
@@ -245,15 +278,35 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
             const int lane = vp / L::WPL, u = vp % L::WPL;
             const int co = lane & 15, th = lane >> 4;
             const int j = co * CPL / 32;
+            // TPW tokens x CPL channels: per token one threshold triple (one
+            // 8-byte load) and CPL/2 channel pairs (CPL/8 16-byte loads).
+            uint32_t x[8], b1[TPW], b2[TPW], b3[TPW];
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt) {
+                const int t = 16 * th + u * TPW + tt;
+                const uint2 tr = *(const uint2 *)(thrV + (t * NJ + j) * 4);
+                b1[tt] = __byte_perm(tr.x, 0, 0x1010);
+                b2[tt] = __byte_perm(tr.x, 0, 0x3232);
+                b3[tt] = __byte_perm(tr.y, 0, 0x1010);
+                const uint16_t *row = tv + t * RS + co * CPL;
+                if constexpr (CPL >= 8) {
+#pragma unroll
+                    for (int v = 0; v < CPL / 8; ++v) {
+                        const uint4 a = *(const uint4 *)(row + 8 * v);
+                        const int i0 = tt * (CPL / 2) + 4 * v;
+                        x[i0] = a.x; x[i0 + 1] = a.y; x[i0 + 2] = a.z; x[i0 + 3] = a.w;
+                    }
+                } else {
+                    const uint2 a = *(const uint2 *)row;
+                    x[tt * 2] = a.x;
+                    x[tt * 2 + 1] = a.y;
+                }
+            }
             uint32_t word = 0;
 #pragma unroll
             for (int i = 7; i >= 0; --i) {
-                const int tt = i / (CPL / 2), m = i % (CPL / 2);
-                const int t = 16 * th + u * TPW + tt;
-                const uint16_t *tr = thrV + (t * NJ + j) * 4;
-                const uint32_t b1 = tr[0], b2 = tr[1], b3 = tr[2];
-                const uint32_t x = *(const uint32_t *)(tv + t * RS + co * CPL + 2 * m);
-                word = word * 4u + code_pair_bits<DT>(x, b1 | (b1 << 16), b2 | (b2 << 16), b3 | (b3 << 16));
+                const int tt = i / (CPL / 2);
+                word = word * 4u + code_pair_bits<DT>(x[i], b1[tt], b2[tt], b3[tt]);
             }
             *(uint32_t *)(outb + L::VC + code_word_offset(lane, u)) = word;
         }
