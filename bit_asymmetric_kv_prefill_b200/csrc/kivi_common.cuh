@@ -98,12 +98,15 @@ __host__ __device__ inline int km_offset(int P)
 // the definition code = clamp(rint(fl(fl(x - z) / s)), 0, 3) (fp32, rint half
 // to even) equals [d > E1] + [d > E2] + [d > E3] with d = fl(x - z), because
 // division and rounding are monotone:
-//   rint(y) >= 1  <=> y > 0.5          <=> d/s > 0.5 + 2^-25  (tie -> 0.5)
-//   rint(y) >= 2  <=> y >= 1.5         <=> d/s >= 1.5 - 2^-24 (tie -> 1.5)
-//   rint(y) >= 3  <=> y > 2.5          <=> d/s > 2.5 + 2^-23  (tie -> 2.5)
-// Each bound times s is exact in double (<= 37 significant bits); a strict
-// fp32 threshold E with d > E <=> d > X is RD(X), and for d >= X it is
-// pred(RU(X)).  A zero scale gives thresholds +inf (all codes 0).
+//   rint(y) >= 1  <=> y > 0.5   <=> d/s > 0.5 + 2^-25  (a tie rounds to 0.5)
+//   rint(y) >= 2  <=> y >= 1.5  <=> d/s >= 1.5 - 2^-24 (a tie rounds to 1.5)
+//   rint(y) >= 3  <=> y > 2.5   <=> d/s > 2.5 + 2^-23  (a tie rounds to 2.5)
+// s has at most 11 significant bits, so s/2, 1.5s and 2.5s are exact in fp32,
+// and each bound times s lies strictly inside one fp32 ulp next to them
+// ((0.5 + 2^-25)s in (s/2, succ(s/2)), (1.5 - 2^-24)s in (pred(1.5s), 1.5s),
+// (2.5 + 2^-23)s in (2.5s, succ(2.5s))).  For an fp32 d the three tests are
+// therefore d > s/2, d > pred(1.5s) and d > 2.5s.  A zero scale gives
+// thresholds +inf (all codes 0).
 // ---------------------------------------------------------------------------
 struct CodeParams {
     uint16_t s_bits, z_bits;
@@ -126,13 +129,9 @@ __device__ __forceinline__ CodeParams code_params(float mn, float mx)
     if (sf == 0.0f) {
         p.e1 = p.e2 = p.e3 = __int_as_float(0x7f800000);
     } else {
-        double s = (double)sf;
-        double x1 = (0.5 + 0x1p-25) * s;
-        double x2 = (1.5 - 0x1p-24) * s;
-        double x3 = (2.5 + 0x1p-23) * s;
-        p.e1 = __double2float_rd(x1);
-        p.e2 = __int_as_float(__float_as_int(__double2float_ru(x2)) - 1);
-        p.e3 = __double2float_rd(x3);
+        p.e1 = __fmul_rn(sf, 0.5f);
+        p.e2 = __int_as_float(__float_as_int(__fmul_rn(sf, 1.5f)) - 1);
+        p.e3 = __fmul_rn(sf, 2.5f);
     }
     return p;
 }

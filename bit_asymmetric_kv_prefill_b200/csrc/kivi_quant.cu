@@ -38,7 +38,7 @@ template <>
 struct In<1> {  // bfloat16
     static constexpr uint16_t kInf = 0x7F80u, kNegInf = 0xFF80u;
     __device__ static float f(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
-    __device__ static uint16_t from_double(double y) { return __bfloat16_as_ushort(__double2bfloat16(y)); }
+    __device__ static uint16_t from_float_rd(float y) { return __bfloat16_as_ushort(__float2bfloat16_rd(y)); }
     __device__ static __nv_bfloat162 v(uint32_t u)
     {
         __nv_bfloat162 r;
@@ -60,7 +60,7 @@ template <>
 struct In<0> {  // IEEE fp16
     static constexpr uint16_t kInf = 0x7C00u, kNegInf = 0xFC00u;
     __device__ static float f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
-    __device__ static uint16_t from_double(double y) { return __half_as_ushort(__double2half(y)); }
+    __device__ static uint16_t from_float_rd(float y) { return __half_as_ushort(__float2half_rd(y)); }
     __device__ static __half2 v(uint32_t u)
     {
         __half2 r;
@@ -104,23 +104,33 @@ __device__ __forceinline__ bool passes(uint16_t x, float e, float z)
 }
 
 // Smallest input value x (as bits) with fl32(x - z) > e; +inf when none.
-// fl32(x - z) is non-decreasing in x, so {x : passes} is an upper set; the
-// start point rounds z + e to the input dtype and a few bounded steps settle
-// on its least element.
+// fl32(x - z) is non-decreasing in x, so {x : passes} is an upper set.  The
+// start c = RD_dtype(RD_fp32(z + e)) satisfies c - z <= e, so it never
+// passes; stepping up reaches the least passing value, normally in one or two
+// steps.  Should that not happen within 4 steps, a binary search over the
+// value-ordered 16-bit patterns settles it.
 template <int DT>
 __device__ __forceinline__ uint16_t min_passing(float e, float z)
 {
     if (!(e < __int_as_float(0x7f800000))) return In<DT>::kInf;
-    uint16_t x = In<DT>::from_double((double)e + (double)z);
+    uint16_t x = In<DT>::from_float_rd(__fadd_rd(z, e));
 #pragma unroll 1
-    for (int i = 0; i < 8; ++i) {
-        const uint16_t d = next_down<DT>(x);
-        if (d == x || !passes<DT>(d, e, z)) break;
-        x = d;
+    for (int i = 0; i < 4; ++i) {
+        x = next_up<DT>(x);
+        if (passes<DT>(x, e, z)) return x;
     }
+    // Value-order key of a pattern: negatives reversed below the positives.
+    auto key_bits = [](int k) -> uint16_t {
+        return k < 0x8000 ? (uint16_t)(0xffff - k) : (uint16_t)(k - 0x8000);
+    };
+    int lo = 0x8000 - (In<DT>::kInf & 0x7fff), hi = 0x8000 + In<DT>::kInf;  // -inf .. +inf
 #pragma unroll 1
-    for (int i = 0; i < 8 && !passes<DT>(x, e, z); ++i) x = next_up<DT>(x);
-    return x;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (passes<DT>(key_bits(mid), e, z)) hi = mid;
+        else lo = mid + 1;
+    }
+    return key_bits(lo);
 }
 
 // Two codes of a channel pair x (packed) against packed thresholds t1..t3:
