@@ -153,6 +153,14 @@ __device__ __forceinline__ uint32_t code_of(float x, float z, float e1, float e2
 // last(s) - first(s) + 1 partials, first(s) = owner(s*C),
 // last(s) = owner((s+1)*C - 1).
 // ---------------------------------------------------------------------------
+// floor(a / b) for 0 <= a < 2^53, b >= 1, exactly: the double quotient is
+// correctly rounded and a non-integer a/b sits at least 1/b away from both
+// neighbouring integers, farther than the rounding error (a/b)*2^-53.
+__host__ __device__ __forceinline__ long long floor_div(long long a, long long b)
+{
+    return (long long)((double)a / (double)b);
+}
+
 struct Split {
     long long seqs, n_groups, n_res_items, C, Tot, warps;
     int wg, wr;
@@ -170,10 +178,10 @@ struct Split {
         warps = warps_;
     }
     __host__ __device__ long long n_items() const { return n_groups + n_res_items; }
-    __host__ __device__ long long lo(long long w) const { return w * Tot / warps; }
+    __host__ __device__ long long lo(long long w) const { return floor_div(w * Tot, warps); }
     __host__ __device__ long long owner(long long pos) const
     {
-        return ((pos + 1) * warps - 1) / Tot;
+        return floor_div((pos + 1) * warps - 1, Tot);
     }
     __host__ __device__ long long item_start(long long idx) const
     {
@@ -184,9 +192,9 @@ struct Split {
     __host__ __device__ long long first_item_at(long long rel) const
     {
         long long gend = n_groups * wg;
-        if (n_groups > 0 && rel <= gend - wg) return (rel + wg - 1) / wg;
+        if (n_groups > 0 && rel <= gend - wg) return floor_div(rel + wg - 1, wg);
         if (rel <= gend) return n_groups;
-        long long idx = n_groups + (rel - gend + wr - 1) / wr;
+        long long idx = n_groups + floor_div(rel - gend + wr - 1, wr);
         return idx < n_items() ? idx : n_items();
     }
     // Items of sequence s owned by warp w: [*i0, *i1).

@@ -215,7 +215,20 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     Split sp;
     sp.init(p.seqs, p.n_groups, p.r, p.wg, p.wr, p.warps);
     const long long lo = sp.lo(gw), hi = sp.lo(gw + 1);
-    const long long s_first = lo / sp.C, s_last = (hi - 1) / sp.C;
+    const long long s_first = floor_div(lo, sp.C), s_last = floor_div(hi - 1, sp.C);
+
+    // The query rows of the warp's next sequence travel in registers ahead of
+    // use (packed pairs of the cache dtype), starting with the first one.
+    constexpr int QW = HG * D / 64;
+    uint32_t qnext[QW];
+    auto load_q = [&](long long s) {
+        const long long b = floor_div(s, p.H_kv);
+        const int hk = (int)(s - b * p.H_kv);
+        const uint32_t *qg = (const uint32_t *)(p.q + (b * p.H_q + (long long)hk * HG) * D);
+#pragma unroll
+        for (int i = 0; i < QW; ++i) qnext[i] = __ldg(qg + lane + 32 * i);
+    };
+    load_q(s_first);
 
     if (lane == 0) {
         for (int i = 0; i < kStages; ++i) mbar_init(bar0 + 8 * i, 1);
@@ -290,14 +303,22 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     for (long long s = s_first; s <= s_last && !failed; ++s) {
         long long i0, i1;
         sp.items(s, gw, &i0, &i1);
-        const long long b = s / p.H_kv;
-        const int hk = (int)(s % p.H_kv);
-        const uint16_t *qg = p.q + (b * p.H_q + (long long)hk * HG) * D;
+        const long long b = floor_div(s, p.H_kv);
+        const int hk = (int)(s - b * p.H_kv);
 
-        // Scaled query in shared memory (fp32) and the lane's q' inputs.
+        // Scaled query in shared memory (fp32) and the lane's q' inputs; then
+        // the next sequence's query is requested (with four or more query
+        // heads per group the registers are short: those load in place).
+        if (HG > 2 && s != s_first) load_q(s);
         __syncwarp();
-        for (int i = lane; i < HG * D; i += 32) qs[i] = to_f<DT>(qg[i]) * p.qscale;
+#pragma unroll
+        for (int i = 0; i < QW; ++i) {
+            const int e = 2 * (lane + 32 * i);
+            qs[e] = to_f<DT>((uint16_t)qnext[i]) * p.qscale;
+            qs[e + 1] = to_f<DT>((uint16_t)(qnext[i] >> 16)) * p.qscale;
+        }
         __syncwarp();
+        if (HG <= 2 && s < s_last) load_q(s + 1);
         float qreg[HG][QPL], qsc[HG][QPL];
 #pragma unroll
         for (int h = 0; h < HG; ++h)
@@ -683,7 +704,9 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         is_last = __shfl_sync(FULL, is_last, 0);
         if (!is_last) continue;
         __threadfence();
-        // Log-sum-exp merge of the `count` partials of sequence s.
+        // Log-sum-exp merge of the `count` partials of sequence s: lanes load
+        // the (m, l) of 32 partials at a time, then every lane streams its
+        // channels of all partials with independent loads.
 #pragma unroll 1
         for (int h = 0; h < HG; ++h) {
             float mx = -INFINITY;
@@ -694,20 +717,28 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
             float oo[QPL];
 #pragma unroll
             for (int c = 0; c < QPL; ++c) oo[c] = 0.f;
-#pragma unroll 4
-            for (int k = 0; k < count; ++k) {
-                const float *pk = pbase + ((long long)k * HG + h) * PSTRIDE;
-                const float2 ml = __ldcg((const float2 *)(pk + D));
-                const float wgt = ex2(ml.x - mx);
-                lacc = fmaf(wgt, ml.y, lacc);
+            for (int k0 = 0; k0 < count; k0 += 32) {
+                const int kk = k0 + lane;
+                float wk = 0.f;
+                if (kk < count) {
+                    const float2 ml = __ldcg((const float2 *)(pbase + ((long long)kk * HG + h) * PSTRIDE + D));
+                    wk = ex2(ml.x - mx);
+                    lacc = fmaf(wk, ml.y, lacc);
+                }
+                const int n = min(32, count - k0);
+#pragma unroll 8
+                for (int j = 0; j < n; ++j) {
+                    const float wj = __shfl_sync(FULL, wk, j);
+                    const float *pk = pbase + ((long long)(k0 + j) * HG + h) * PSTRIDE + lane * QPL;
 #pragma unroll
-                for (int c = 0; c < QPL; c += 2) {
-                    const float2 v = __ldcg((const float2 *)(pk + lane * QPL + c));
-                    oo[c] = fmaf(wgt, v.x, oo[c]);
-                    oo[c + 1] = fmaf(wgt, v.y, oo[c + 1]);
+                    for (int c = 0; c < QPL; c += 2) {
+                        const float2 v = __ldcg((const float2 *)(pk + c));
+                        oo[c] = fmaf(wj, v.x, oo[c]);
+                        oo[c + 1] = fmaf(wj, v.y, oo[c + 1]);
+                    }
                 }
             }
-            const float inv = 1.0f / lacc;
+            const float inv = 1.0f / warp_sum(lacc);
 #pragma unroll
             for (int c = 0; c < QPL; c += 2)
                 *(float2 *)(outrow + h * D + lane * QPL + c) = make_float2(oo[c] * inv, oo[c + 1] * inv);
