@@ -45,6 +45,9 @@ namespace kivi {
 #ifndef KIVI_DECODE_MAXW
 #define KIVI_DECODE_MAXW 16
 #endif
+#ifndef KIVI_DECODE_MAXW_GQA
+#define KIVI_DECODE_MAXW_GQA 12   // four or more query heads per kv head
+#endif
 #ifndef KIVI_SCALAR_F32
 #define KIVI_SCALAR_F32 0
 #endif
@@ -141,6 +144,43 @@ __device__ __forceinline__ float2 code_pair(uint32_t w, uint32_t w16, int i, uin
 }
 // 2^-2i, the inverse of pair i's shift.
 __device__ __forceinline__ float pair_scale(int i) { return __uint_as_float((uint32_t)(127 - 2 * i) << 23); }
+// 2^e for -126 <= e <= 127.
+__device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
+
+// Keys, fast path: AND-ing pair i's field out of the word (or of the word
+// shifted right by 16) leaves the fp32 denormal c * 2^(2i-149).  Multiplying
+// by q'' = q' * 2^(kKexp-2i) gives q' c 2^(kKexp-149) with no conversion
+// step; one logic op per code and one fp32x2 FMA per pair.
+constexpr int kKexp = 64;
+constexpr float kKunscale = 0x1p85f;   // 2^(149 - kKexp)
+__device__ __forceinline__ float kq_scale(int i) { return pow2i(kKexp - 2 * i); }
+
+// Values: AND-ing 0x00030003 << 2j out of a word leaves two f16 subnormals
+// c * 2^(2j-24) in its halves (j <= 3; pairs 4..7 are read from the word
+// shifted right by 8).  They multiply an f16 token weight in a mixed-precision
+// FMA (exact f16 products, fp32 accumulation).  HA/HB pick the halves.
+template <int HA, int HB>
+__device__ __forceinline__ float hfma_f32(uint32_t a, uint32_t b, float c)
+{
+    float d;
+    if constexpr (HA == 0 && HB == 0)
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.f16 %0, a0, b0, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else if constexpr (HA == 1 && HB == 0)
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.f16 %0, a1, b0, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else if constexpr (HA == 0 && HB == 1)
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.f16 %0, a0, b1, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    else
+        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+            "fma.rn.f32.f16 %0, a1, b1, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+// Token weights are kept near 2^6 on the first group (room for the 2^8 of
+// softmax slack below the f16 limit) and scaled down when one would pass 2^15.
+constexpr int kVTargetExp = 6;
+constexpr float kVLimit = 32768.0f;
 
 template <int DT>
 __device__ __forceinline__ float to_f(uint16_t b)
@@ -168,11 +208,11 @@ template <int D, int HG, bool ROPE>
 struct WarpSmem {
     using L = Layout<D>;
     static constexpr int QPS = D / 4 + 4;           // padded q' slice (floats)
-    static constexpr int PPS = 34;                  // padded p' row (float2)
+    static constexpr int PPS = 40;                  // padded weight row (f16)
     static constexpr int RING = 0;                  // kStages x GB
     static constexpr int QP = kStages * L::GB;      // float [HG][4][QPS]
-    static constexpr int PP = QP + HG * 4 * QPS * 4;          // float2 [HG][NJ][PPS]
-    static constexpr int QS = PP + HG * L::NJ * PPS * 8;      // float [HG][D]
+    static constexpr int PP = QP + HG * 4 * QPS * 4;          // f16 [HG][NJ][PPS]
+    static constexpr int QS = PP + HG * L::NJ * PPS * 2;      // float [HG][D]
     static constexpr int SZ = QS + HG * D * 4;                // float2 [4][D/4] (RoPE)
     static constexpr int BAR = SZ + (ROPE ? D * 8 : 0);       // uint64 [kStages]
     static constexpr int BYTES = (BAR + kStages * 8 + 15) / 16 * 16;
@@ -182,7 +222,8 @@ template <int D, int HG, bool ROPE>
 struct DecodeShape {
     static constexpr int PER_WARP = WarpSmem<D, HG, ROPE>::BYTES;
     static constexpr int MAXW = 232448 / PER_WARP;
-    static constexpr int NW = MAXW > KIVI_DECODE_MAXW ? KIVI_DECODE_MAXW : MAXW;
+    static constexpr int CAP = HG >= 4 ? KIVI_DECODE_MAXW_GQA : KIVI_DECODE_MAXW;
+    static constexpr int NW = MAXW > CAP ? CAP : MAXW;
     static constexpr int SMEM = NW * PER_WARP;
 };
 
@@ -205,7 +246,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     unsigned char *ws = smem_all + warp * W::BYTES;
     unsigned char *ring = ws + W::RING;
     float *qp = (float *)(ws + W::QP);
-    float2 *pp = (float2 *)(ws + W::PP);
+    uint16_t *pp = (uint16_t *)(ws + W::PP);
     float *qs = (float *)(ws + W::QS);
     float2 *sz = (float2 *)(ws + W::SZ);
     const uint32_t bar0 = smem_addr(ws + W::BAR);
@@ -297,8 +338,9 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     const int pL0 = (lane & 7) * QPL;           //   and first local index
     const int vco = lane & 15, vth = lane >> 4; // V mapping: channel octet, token half
     const int jl = vco * CPL / 32;              //   value group of the lane's channels
-    // V: token factor 2^(-CPL*(t mod TPW)) of token t = lane.
-    const float vtok = __uint_as_float((uint32_t)(127 - CPL * (lane % TPW)) << 23);
+    // V: token t = lane's weight factor undoing the shift its pairs are read
+    // at, 2^-(2*((t mod TPW)*CPL/2 mod 4)).
+    const float vtok = pow2i(-2 * (((lane % TPW) * (CPL / 2)) & 3));
 
     for (long long s = s_first; s <= s_last && !failed; ++s) {
         long long i0, i1;
@@ -325,13 +367,18 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
 #pragma unroll
             for (int e = 0; e < QPL; ++e) {
                 qreg[h][e] = qs[h * D + k_channel<D>(pcs, pL0 + e)];
-                qsc[h][e] = qreg[h][e] * pair_scale(((pL0 + e) & 15) >> 1);
+                qsc[h][e] = qreg[h][e] * (ROPE ? pair_scale(((pL0 + e) & 15) >> 1) : kq_scale(((pL0 + e) & 15) >> 1));
             }
 
         float m[HG], lsum[HG], zacc[HG][NJ];
         float2 accV[HG][CPL / 2];
+        // accV[h][mm] holds sum_t p_t s_t c_t 2^(2mm-24) * 2^ev[h].
+        int ev[HG];
+        bool ev_fresh[HG];
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
+            ev[h] = 0;
+            ev_fresh[h] = true;
             m[h] = -INFINITY;
             lsum[h] = 0.f;
 #pragma unroll
@@ -435,8 +482,10 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
 #pragma unroll
                             for (int t = 0; t < 4; ++t) {
                                 const uint32_t w = kw[t * KW + k];
-                                const float2 c01 = code_pair(w, kw16[t], i / 2, magic, neg);
-                                const float2 c23 = code_pair(w, kw16[t], i / 2 + 1, magic, neg);
+                                const float2 c01 = make_float2(__uint_as_float(w & (3u << i)),
+                                                               __uint_as_float(kw16[t] & (3u << i)));
+                                const float2 c23 = make_float2(__uint_as_float(w & (12u << i)),
+                                                               __uint_as_float(kw16[t] & (12u << i)));
 #pragma unroll
                                 for (int h = 0; h < HG; ++h) {
                                     acc[t][h] = ffma2(make_float2(q4[h].x, q4[h].y), c01, acc[t][h]);
@@ -502,23 +551,53 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     float send = loB ? k0 : k1;
                     float keep = (loB ? k1 : k0) + __shfl_xor_sync(FULL, send, 1);
                     if constexpr (ROPE) sc[h] = keep;
-                    else sc[h] = keep + bias[h];
+                    else sc[h] = fmaf(keep, kKunscale, bias[h]);
                 }
                 float pr[HG];
                 softmax_step(sc, pr, true);
 
-                // Value scales for token `lane`; p' carries the token's
-                // power-of-two factor of the fast code path.
+                // Token weights b = p s 2^ev (times the lane's shift factor)
+                // for token `lane`, as f16 rows [h][j][token].
                 const uint16_t *vm = (const uint16_t *)(st + L::VM + lane * (D / 8));
+                float svj[NJ];
 #pragma unroll
                 for (int j = 0; j < NJ; ++j) {
-                    const float svj = f16f(vm[j]) * vtok, zvj = f16f(vm[NJ + j]);
+                    svj[j] = f16f(vm[j]) * vtok;
+                    const float zvj = f16f(vm[NJ + j]);
 #pragma unroll
-                    for (int h = 0; h < HG; ++h) {
-                        const float pv = pr[h] * svj;
-                        pp[(h * NJ + j) * W::PPS + lane] = make_float2(pv, pv);
-                        zacc[h][j] = fmaf(pr[h], zvj, zacc[h][j]);
+                    for (int h = 0; h < HG; ++h) zacc[h][j] = fmaf(pr[h], zvj, zacc[h][j]);
+                }
+#pragma unroll
+                for (int h = 0; h < HG; ++h) {
+                    float f = pr[h] * pow2i(ev[h]);
+                    float bm = 0.f;
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j) bm = fmaxf(bm, f * svj[j]);
+                    if (__any_sync(FULL, !(bm < kVLimit)) || ev_fresh[h]) {
+                        // Rare: choose 2^d putting the largest weight near
+                        // kVTarget (first group with a nonzero weight), or
+                        // bring it below the f16 range; accV follows.
+                        const float mx = warp_max(bm);
+                        if (mx > 0.f && mx <= 3.0e38f) {
+                            const int e = (int)((__float_as_uint(mx) >> 23) & 0xff) - 127;
+                            int d = kVTargetExp - e;
+                            if (!ev_fresh[h] && d > 0) d = 0;
+                            const int en = max(-100, min(100, ev[h] + d));
+                            d = en - ev[h];
+                            const int d1 = d / 2, d2 = d - d1;
+#pragma unroll
+                            for (int c = 0; c < CPL / 2; ++c) {
+                                accV[h][c].x = accV[h][c].x * pow2i(d1) * pow2i(d2);
+                                accV[h][c].y = accV[h][c].y * pow2i(d1) * pow2i(d2);
+                            }
+                            f = pr[h] * pow2i(en);
+                            ev[h] = en;
+                            ev_fresh[h] = false;
+                        }
                     }
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j)
+                        pp[(h * NJ + j) * W::PPS + lane] = __half_as_ushort(__float2half_rn(f * svj[j]));
                 }
                 __syncwarp();
 
@@ -533,25 +612,33 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     vw[4 * c + 2] = v4.z;
                     vw[4 * c + 3] = v4.w;
                 }
+                // The 16 token weights of the lane's tokens, two per word.
+                uint32_t pb[HG][8];
+#pragma unroll
+                for (int h = 0; h < HG; ++h) {
+                    const uint4 *src = (const uint4 *)(pp + (h * NJ + jl) * W::PPS + 16 * vth);
+                    const uint4 a = src[0], b = src[1];
+                    pb[h][0] = a.x; pb[h][1] = a.y; pb[h][2] = a.z; pb[h][3] = a.w;
+                    pb[h][4] = b.x; pb[h][5] = b.y; pb[h][6] = b.z; pb[h][7] = b.w;
+                }
 #pragma unroll
                 for (int u = 0; u < L::WPL; ++u) {
-                    const uint32_t w = vw[u], w16 = w >> 16;
+                    const uint32_t w = vw[u], w8 = w >> 8;
 #pragma unroll
-                    for (int t2 = 0; t2 < TPW; t2 += 2) {
-                        float4 p4[HG];
+                    for (int tt = 0; tt < TPW; ++tt) {
 #pragma unroll
-                        for (int h = 0; h < HG; ++h)
-                            p4[h] = *(const float4 *)(pp + (h * NJ + jl) * W::PPS + 16 * vth + u * TPW + t2);
+                        for (int mm = 0; mm < CPL / 2; ++mm) {
+                            const int i = tt * (CPL / 2) + mm;
+                            const uint32_t x = (i < 4 ? w : w8) & (0x00030003u << (2 * (i & 3)));
 #pragma unroll
-                        for (int tt = 0; tt < 2; ++tt) {
-#pragma unroll
-                            for (int mm = 0; mm < CPL / 2; ++mm) {
-                                const float2 cc = code_pair(w, w16, (t2 + tt) * (CPL / 2) + mm, magic, neg);
-#pragma unroll
-                                for (int h = 0; h < HG; ++h) {
-                                    const float2 pv = tt == 0 ? make_float2(p4[h].x, p4[h].y)
-                                                              : make_float2(p4[h].z, p4[h].w);
-                                    accV[h][mm] = ffma2(pv, cc, accV[h][mm]);
+                            for (int h = 0; h < HG; ++h) {
+                                const uint32_t bw = pb[h][(u * TPW + tt) >> 1];
+                                if ((tt & 1) == 0) {
+                                    accV[h][mm].x = hfma_f32<0, 0>(x, bw, accV[h][mm].x);
+                                    accV[h][mm].y = hfma_f32<1, 0>(x, bw, accV[h][mm].y);
+                                } else {
+                                    accV[h][mm].x = hfma_f32<0, 1>(x, bw, accV[h][mm].x);
+                                    accV[h][mm].y = hfma_f32<1, 1>(x, bw, accV[h][mm].y);
                                 }
                             }
                         }
@@ -622,18 +709,20 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     if (ok) {
                         const uint16_t *vrow = rv + t * D + vco * CPL;
 #pragma unroll
-                        for (int c = 0; c < CPL; ++c) vx[c] = to_f<DT>(vrow[c]) * (float)(1 << (2 * (c / 2)));
+                        for (int c = 0; c < CPL; ++c) vx[c] = to_f<DT>(vrow[c]);
                     } else {
 #pragma unroll
                         for (int c = 0; c < CPL; ++c) vx[c] = 0.f;
                     }
 #pragma unroll
                     for (int h = 0; h < HG; ++h) {
-                        const float pt = __shfl_sync(FULL, pr[h], 4 * (ok ? t : t0));
+                        const float pt = __shfl_sync(FULL, pr[h], 4 * (ok ? t : t0)) * pow2i(ev[h] - 24);
 #pragma unroll
-                        for (int c = 0; c < CPL; c += 2)
-                            accV[h][c / 2] = ffma2(make_float2(pt, pt), make_float2(vx[c], vx[c + 1]),
+                        for (int c = 0; c < CPL; c += 2) {
+                            const float pa = pt * pow2i(c);   // 2^(2mm), mm = c/2
+                            accV[h][c / 2] = ffma2(make_float2(pa, pa), make_float2(vx[c], vx[c + 1]),
                                                    accV[h][c / 2]);
+                        }
                     }
                 }
             }
@@ -664,7 +753,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
 #pragma unroll
             for (int c = 0; c < CPL; c += 2) {
                 const float2 a = accV[h][c / 2];
-                const float f = 1.0f / (float)(1 << (2 * (c / 2)));
+                const float f = pow2i(24 - c - ev[h]);   // 2^(24 - 2mm - ev)
                 const float x = a.x + __shfl_xor_sync(FULL, a.x, 16);
                 const float y = a.y + __shfl_xor_sync(FULL, a.y, 16);
                 o[h][c] = fmaf(x, f, zt[h][jl]);

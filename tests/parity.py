@@ -120,3 +120,37 @@ class Pair:
                 for key in ref:
                     if not np.array_equal(got[key][0], ref[key][i, 0]):
                         raise AssertionError(f"{key} differs for sequence {s}")
+
+
+def _vals(bits, dtype):
+    bits = np.asarray(bits, np.uint16)
+    if dtype == "bf16":
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return bits.view(np.float16).astype(np.float64)
+
+
+def value_weight_bound(cache: KiviCache, q_bits, w: synth.Workload):
+    """Elementwise bound on |decode - oracle| from the one rounding the decode
+    kernel adds to fp32 accumulation: each quantized token's value weight
+    p_t * s_t enters the code product as an f16 (relative error <= 2^-11), so
+    |d o_c| <= 2^-11 * sum_t w_t s_t c_t,c with w the softmax weights.  Float64
+    attention over the exported cache (no pre-RoPE keys)."""
+    assert not w.pre_rope
+    a = cache.export()
+    n_q, r = cache.length()
+    D, G, HG = w.D, w.G, w.H_q // w.H_kv
+    q = _vals(q_bits, w.dtype)
+    bound = np.zeros((w.B, w.H_q, D))
+    for s in range(w.B * w.H_kv):
+        b, hk = divmod(s, w.H_kv)
+        sK = np.repeat(_vals(a["sK"][s], "fp16"), G, axis=0)[:n_q]
+        zK = np.repeat(_vals(a["zK"][s], "fp16"), G, axis=0)[:n_q]
+        keys = np.concatenate([a["codesK"][s] * sK + zK, _vals(a["resK"][s], w.dtype)])
+        sV = np.repeat(_vals(a["sV"][s], "fp16"), G, axis=1)       # [n_q, D]
+        for g in range(HG):
+            h = hk * HG + g
+            sc = keys @ q[b, h] / np.sqrt(D)
+            p = np.exp(sc - sc.max())
+            p /= p.sum()
+            bound[b, h] = 2.0 ** -11 * (p[:n_q, None] * sV * a["codesV"][s]).sum(axis=0)
+    return bound
