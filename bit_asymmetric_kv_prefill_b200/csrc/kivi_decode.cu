@@ -55,7 +55,7 @@ namespace kivi {
 constexpr unsigned FULL = 0xffffffffu;
 constexpr int kStages = KIVI_DECODE_STAGES;
 constexpr float kRescaleSlack = 8.0f;
-constexpr long long kWaitLimit = 1LL << 22;
+constexpr int kWaitLimit = 1 << 22;
 
 // ---- PTX wrappers ----------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
@@ -90,6 +90,27 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
             dst),
         "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+// Lane 0 of the calling warp arms `bar` for `bytes` and starts one bulk copy
+// of `bytes` into it; the other lanes skip both under a predicate (no branch).
+__device__ __forceinline__ void lane0_expect_copy(int lane, uint32_t bar, uint32_t dst, const void *src,
+                                                  uint32_t bytes, uint32_t expect)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, %0, 0;\n\t"
+        "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %5;\n\t"
+        "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%2], [%3], %4, [%1];\n\t}"
+        ::"r"(lane), "r"(bar), "r"(dst), "l"(src), "r"(bytes), "r"(expect)
+        : "memory");
+}
+__device__ __forceinline__ void lane0_copy(int lane, uint32_t bar, uint32_t dst, const void *src,
+                                           uint32_t bytes)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, %0, 0;\n\t"
+        "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%2], [%3], %4, [%1];\n\t}"
+        ::"r"(lane), "r"(bar), "r"(dst), "l"(src), "r"(bytes)
         : "memory");
 }
 __device__ __forceinline__ float ex2(float x)
@@ -253,19 +274,35 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     const uint32_t magic = p.magic;
     const float2 neg = make_float2(p.neg_magic, p.neg_magic);
 
+    // This warp's share of the flattened (sequence, item) list: sequences
+    // s_first..s_last, items [i_first, ...) of the first and [..., i_end) of
+    // the last; the sequences between are whole.  Item indices fit 32 bits.
     Split sp;
     sp.init(p.seqs, p.n_groups, p.r, p.wg, p.wr, p.warps);
     const long long lo = sp.lo(gw), hi = sp.lo(gw + 1);
-    const long long s_first = floor_div(lo, sp.C), s_last = floor_div(hi - 1, sp.C);
+    const int s_first = (int)floor_div(lo, sp.C), s_last = (int)floor_div(hi - 1, sp.C);
+    const int n_items = (int)sp.n_items(), n_groups = (int)p.n_groups;
+    int i_first, i_end;
+    {
+        long long a0, a1, b0, b1;
+        sp.items(s_first, gw, &a0, &a1);
+        sp.items(s_last, gw, &b0, &b1);
+        i_first = (int)a0;
+        i_end = (int)b1;
+    }
+    auto seq_items = [&](int s, int *i0, int *i1) {
+        *i0 = s == s_first ? i_first : 0;
+        *i1 = s == s_last ? i_end : n_items;
+        if (*i1 < *i0) *i1 = *i0;
+    };
 
     // The query rows of the warp's next sequence travel in registers ahead of
     // use (packed pairs of the cache dtype), starting with the first one.
     constexpr int QW = HG * D / 64;
     uint32_t qnext[QW];
-    auto load_q = [&](long long s) {
-        const long long b = floor_div(s, p.H_kv);
-        const int hk = (int)(s - b * p.H_kv);
-        const uint32_t *qg = (const uint32_t *)(p.q + (b * p.H_q + (long long)hk * HG) * D);
+    auto load_q = [&](int s) {
+        const int b = s / p.H_kv, hk = s - b * p.H_kv;
+        const uint32_t *qg = (const uint32_t *)(p.q + ((long long)b * p.H_q + (long long)hk * HG) * D);
 #pragma unroll
         for (int i = 0; i < QW; ++i) qnext[i] = __ldg(qg + lane + 32 * i);
     };
@@ -278,12 +315,12 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     __syncwarp();
 
     // Prefetch iterator over the warp's items, possibly across sequences.
-    long long pf_s = s_first, pf_i = 0, pf_e = 0;
-    sp.items(pf_s, gw, &pf_i, &pf_e);
+    int pf_s = s_first, pf_i, pf_e;
+    seq_items(pf_s, &pf_i, &pf_e);
     auto pf_advance = [&]() {
         while (pf_i >= pf_e && pf_s < s_last) {
             ++pf_s;
-            sp.items(pf_s, gw, &pf_i, &pf_e);
+            seq_items(pf_s, &pf_i, &pf_e);
         }
     };
     pf_advance();
@@ -291,27 +328,23 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     // and the stage and phase parity of the next item to consume.
     int issued = 0, consumed = 0, ist = 0, cst = 0;
     uint32_t cph = 0;
+    const uint32_t ring_s = smem_addr(ring);
     auto issue_next = [&]() {
         pf_advance();
         if (pf_i >= pf_e) return;
-        const int st = ist;
+        const uint32_t bar = bar0 + 8 * ist;
+        const uint32_t dst = ring_s + ist * L::GB;
         ist = ist + 1 == kStages ? 0 : ist + 1;
-        if (lane == 0) {
-            const uint32_t bar = bar0 + 8 * st;
-            const uint32_t dst = smem_addr(ring + st * L::GB);
-            if (pf_i < p.n_groups) {
-                const uint8_t *src = p.packed + (pf_s * p.ngcap + pf_i) * (long long)L::GB;
-                mbar_expect_tx(bar, L::GB);
-                bulk_g2s(dst, src, L::GB, bar);
-            } else {
-                const int t0 = (int)(pf_i - p.n_groups) * kResTok;
-                const int nt = min(kResTok, p.r - t0);
-                const uint32_t bytes = (uint32_t)nt * D * 2;
-                const long long row = pf_s * (long long)p.R + t0;
-                mbar_expect_tx(bar, 2 * bytes);
-                bulk_g2s(dst, p.resK + row * D, bytes, bar);
-                bulk_g2s(dst + kResTok * D * 2, p.resV + row * D, bytes, bar);
-            }
+        if (pf_i < n_groups) {
+            const uint8_t *src = p.packed + ((long long)pf_s * p.ngcap + pf_i) * (long long)L::GB;
+            lane0_expect_copy(lane, bar, dst, src, L::GB, L::GB);
+        } else {
+            const int t0 = (pf_i - n_groups) * kResTok;
+            const int nt = min(kResTok, p.r - t0);
+            const uint32_t bytes = (uint32_t)nt * D * 2;
+            const long long row = (long long)pf_s * p.R + t0;
+            lane0_expect_copy(lane, bar, dst, p.resK + row * D, bytes, 2 * bytes);
+            lane0_copy(lane, bar, dst + kResTok * D * 2, p.resV + row * D, bytes);
         }
         ++issued;
         ++pf_i;
@@ -321,7 +354,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     bool failed = false;
     auto wait_stage = [&]() -> bool {
         const uint32_t bar = bar0 + 8 * cst;
-        for (long long it = 0; it < kWaitLimit; ++it)
+        for (int it = 0; it < kWaitLimit; ++it)
             if (__all_sync(FULL, mbar_try_wait(bar, cph))) return true;
         return false;
     };
@@ -342,11 +375,10 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     // at, 2^-(2*((t mod TPW)*CPL/2 mod 4)).
     const float vtok = pow2i(-2 * (((lane % TPW) * (CPL / 2)) & 3));
 
-    for (long long s = s_first; s <= s_last && !failed; ++s) {
-        long long i0, i1;
-        sp.items(s, gw, &i0, &i1);
-        const long long b = floor_div(s, p.H_kv);
-        const int hk = (int)(s - b * p.H_kv);
+    for (int s = s_first; s <= s_last && !failed; ++s) {
+        int i0, i1;
+        seq_items(s, &i0, &i1);
+        const int b = s / p.H_kv, hk = s - b * p.H_kv;
 
         // Scaled query in shared memory (fp32) and the lane's q' inputs; then
         // the next sequence's query is requested (with four or more query
@@ -374,10 +406,12 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         float2 accV[HG][CPL / 2];
         // accV[h][mm] holds sum_t p_t s_t c_t 2^(2mm-24) * 2^ev[h].
         int ev[HG];
+        float evs[HG];   // 2^ev
         bool ev_fresh[HG];
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
             ev[h] = 0;
+            evs[h] = 1.0f;
             ev_fresh[h] = true;
             m[h] = -INFINITY;
             lsum[h] = 0.f;
@@ -411,13 +445,13 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
             }
         };
 
-        for (long long it = i0; it < i1; ++it) {
+        for (int it = i0; it < i1; ++it) {
             if (!wait_stage()) {
                 failed = true;
                 break;
             }
             const unsigned char *st = ring + cst * L::GB;
-            if (it < p.n_groups) {
+            if (it < n_groups) {
                 // ---------------- quantized group of 32 tokens ----------------
                 const uint16_t *km = (const uint16_t *)(st + L::KM + lane * (D / 8));
                 float bias[HG];
@@ -500,7 +534,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                         for (int h = 0; h < HG; ++h) part[t][h] = acc[t][h].x + acc[t][h].y;
                 } else {
                     // Dequantize, rotate at absolute positions, dot with q.
-                    const long long tbase = it * kG + 4 * tq;
+                    const long long tbase = (long long)it * kG + 4 * tq;
 #pragma unroll 1
                     for (int t = 0; t < 4; ++t) {
                         float kh[D / 4];
@@ -569,7 +603,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 }
 #pragma unroll
                 for (int h = 0; h < HG; ++h) {
-                    float f = pr[h] * pow2i(ev[h]);
+                    float f = pr[h] * evs[h];
                     float bm = 0.f;
 #pragma unroll
                     for (int j = 0; j < NJ; ++j) bm = fmaxf(bm, f * svj[j]);
@@ -590,7 +624,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                                 accV[h][c].x = accV[h][c].x * pow2i(d1) * pow2i(d2);
                                 accV[h][c].y = accV[h][c].y * pow2i(d1) * pow2i(d2);
                             }
-                            f = pr[h] * pow2i(en);
+                            evs[h] = pow2i(en);
+                            f = pr[h] * evs[h];
                             ev[h] = en;
                             ev_fresh[h] = false;
                         }
@@ -646,7 +681,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 }
             } else {
                 // ---------------- residual slice of up to 6 tokens ----------------
-                const int t0 = (int)(it - p.n_groups) * kResTok;
+                const int t0 = (it - n_groups) * kResTok;
                 const int nt = min(kResTok, p.r - t0);
                 const uint16_t *rk = (const uint16_t *)st;
                 const uint16_t *rv = (const uint16_t *)(st + kResTok * D * 2);
@@ -734,8 +769,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         if (failed) break;
 
         // ---------------- this warp's partial for sequence s ----------------
-        const long long first = sp.owner(s * sp.C);
-        const long long last = sp.owner((s + 1) * sp.C - 1);
+        const long long first = sp.owner((long long)s * sp.C);
+        const long long last = sp.owner(((long long)s + 1) * sp.C - 1);
         const int count = (int)(last - first + 1);
         const int slot = (int)(gw - first);
         float lt[HG], zt[HG][NJ];
@@ -759,7 +794,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 o[h][c] = fmaf(x, f, zt[h][jl]);
                 o[h][c + 1] = fmaf(y, f, zt[h][jl]);
             }
-        float *outrow = p.out + (b * p.H_q + (long long)hk * HG) * D;
+        float *outrow = p.out + ((long long)b * p.H_q + (long long)hk * HG) * D;
         if (count == 1) {
             if (vth == 0) {
 #pragma unroll
@@ -773,7 +808,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
             }
             continue;
         }
-        float *pbase = p.partials + ((s * p.slots) * HG) * (long long)PSTRIDE;
+        float *pbase = p.partials + (((long long)s * p.slots) * HG) * (long long)PSTRIDE;
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
             float *prow = pbase + ((long long)slot * HG + h) * PSTRIDE;
