@@ -328,44 +328,15 @@ kivi_status kivi_append(kivi_cache *c, const void *k_t, const void *v_t, void *s
 
 kivi_status kivi_decode_attn(kivi_cache *c, const void *q, int H_q, float *out, void *stream)
 {
-    if (!c || !q || !out || !aligned16(q) || !aligned16(out)) return KIVI_ERR_ARG;
-    if (!c->prefilled) return KIVI_ERR_STATE;
-    if (H_q < 1 || H_q % c->cfg.H_kv != 0) return KIVI_ERR_ARG;
-    const int HG = H_q / c->cfg.H_kv;
-    const int nw = decode_warps_per_cta(c->cfg.D, HG, c->cfg.pre_rope);
-    if (nw == 0 || HG > kMaxGroupHeads) return KIVI_ERR_UNSUPPORTED;
-    Split sp;
-    sp.init(c->plan.seqs, c->n_q / kG, c->r, c->wg, c->wr, 1);
-    long long warps = (long long)c->sms * nw;
-    if (warps > sp.Tot) warps = sp.Tot;
     DecodeParams p;
-    p.packed = c->packed;
-    p.ngcap = c->plan.ngcap;
-    p.resK = c->resK;
-    p.resV = c->resV;
-    p.R = c->cfg.R;
-    p.q = (const uint16_t *)q;
-    p.out = out;
+    int D = 0, HG = 0, dtype = 0, pre_rope = 0;
+    kivi_status st = decode_params_external_scratch(c, q, H_q, out, &p, &D, &HG, &dtype, &pre_rope);
+    if (st != KIVI_OK) return st;
     p.partials = c->partials;
     p.tickets = c->tickets;
-    p.err = c->err;
-    p.H_kv = c->cfg.H_kv;
-    p.H_q = H_q;
-    p.seqs = c->plan.seqs;
-    p.n_groups = c->n_q / kG;
-    p.r = c->r;
-    p.n_q = c->n_q;
-    p.wg = c->wg;
-    p.wr = c->wr;
-    p.warps = warps;
+    if (p.slots > c->plan.slots) return KIVI_ERR_UNSUPPORTED;
     p.slots = c->plan.slots;
-    p.qscale = (float)(1.4426950408889634 / std::sqrt((double)c->cfg.D));
-    p.inv_freq = c->inv_freq;
-    p.magic = 0x4B000000u;
-    p.neg_magic = -8388608.0f;
-    if (warps / p.seqs + 2 > p.slots) return KIVI_ERR_UNSUPPORTED;
-    cudaError_t e = launch_decode(c->cfg.D, HG, c->cfg.dtype, c->cfg.pre_rope, p,
-                                  (cudaStream_t)stream);
+    cudaError_t e = launch_decode(D, HG, dtype, pre_rope, p, (cudaStream_t)stream);
     return cuda_status(e);
 }
 
@@ -493,6 +464,8 @@ extern "C" kivi_status kivi_decode_split(long long seqs, long long n_groups, int
     sp.init(seqs, n_groups, r, wg, wr, warps);
     if (sp.Tot < 1 || warps > sp.Tot || seq < 0 || seq >= seqs || warp < 0 || warp >= warps)
         return KIVI_ERR_ARG;
+    if ((double)sp.Tot * (double)(warps + 1) >= 9007199254740992.0) return KIVI_ERR_UNSUPPORTED;
+    sp.set_magics();
     out[0] = sp.owner(seq * sp.C);
     out[1] = sp.owner((seq + 1) * sp.C - 1);
     long long i0, i1;
@@ -521,6 +494,16 @@ kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q
     sp.init(c->plan.seqs, c->n_q / kG, c->r, c->wg, c->wr, 1);
     long long warps = (long long)c->sms * nw;
     if (warps > sp.Tot) warps = sp.Tot;
+    sp.init(c->plan.seqs, c->n_q / kG, c->r, c->wg, c->wr, warps);
+    // The split's divisions are exact for numerators below 2^53 (div_floor).
+    if ((double)sp.Tot * (double)(warps + 1) >= 9007199254740992.0) return KIVI_ERR_UNSUPPORTED;
+    sp.set_magics();
+    p->div_C = sp.mC;
+    p->div_Tot = sp.mT;
+    p->div_warps = sp.mW;
+    p->div_wg = sp.mG;
+    p->div_wr = sp.mR;
+    p->div_Hkv = make_magic((unsigned long long)c->cfg.H_kv);
     p->packed = c->packed;
     p->ngcap = c->plan.ngcap;
     p->resK = c->resK;

@@ -153,17 +153,59 @@ __device__ __forceinline__ uint32_t code_of(float x, float z, float e1, float e2
 // last(s) - first(s) + 1 partials, first(s) = owner(s*C),
 // last(s) = owner((s+1)*C - 1).
 // ---------------------------------------------------------------------------
-// floor(a / b) for 0 <= a < 2^53, b >= 1, exactly: the double quotient is
-// correctly rounded and a non-integer a/b sits at least 1/b away from both
-// neighbouring integers, farther than the rounding error (a/b)*2^-53.
-__host__ __device__ __forceinline__ long long floor_div(long long a, long long b)
+// Division by a run-time constant d >= 1 as a multiply and shifts, exact
+// for numerators 0 <= a < 2^53 (Granlund and Montgomery, "Division by
+// invariant integers using multiplication", 1994, round-up method): with
+// l = ceil(log2 d) and M = floor(2^(53+l)/d) + 1, 2^(53+l) < M d <= 2^(53+l) + 2^l,
+// so floor(a/d) = floor(a M / 2^(53+l)).  The product's high word is taken
+// after shifting a left by sa = max(0, 11-l); sb = max(0, l-11) finishes it.
+struct Magic {
+    unsigned long long M;
+    int sa, sb;
+};
+
+__host__ inline Magic make_magic(unsigned long long d)
 {
-    return (long long)((double)a / (double)b);
+    int l = 0;
+    while ((1ULL << l) < d) ++l;
+    Magic m;
+    m.M = (unsigned long long)((((unsigned __int128)1) << (53 + l)) / d) + 1;
+    m.sa = l < 11 ? 11 - l : 0;
+    m.sb = l > 11 ? l - 11 : 0;
+    return m;
+}
+
+__host__ __device__ __forceinline__ unsigned long long mulhi64(unsigned long long a,
+                                                                 unsigned long long b)
+{
+#ifdef __CUDA_ARCH__
+    return __umul64hi(a, b);
+#else
+    return (unsigned long long)(((unsigned __int128)a * b) >> 64);
+#endif
+}
+
+// floor(a / d) for 0 <= a < 2^53, m = make_magic(d).
+__host__ __device__ __forceinline__ long long div_floor(long long a, const Magic &m)
+{
+    return (long long)(mulhi64((unsigned long long)a << m.sa, m.M) >> m.sb);
 }
 
 struct Split {
     long long seqs, n_groups, n_res_items, C, Tot, warps;
     int wg, wr;
+    Magic mC, mT, mW, mG, mR;   // division by C, Tot, warps, wg, wr (div_floor)
+
+    // The division constants, from the host (the kernel takes them from its
+    // parameters).
+    __host__ void set_magics()
+    {
+        mC = make_magic((unsigned long long)C);
+        mT = make_magic((unsigned long long)Tot);
+        mW = make_magic((unsigned long long)warps);
+        mG = make_magic((unsigned long long)wg);
+        mR = make_magic((unsigned long long)wr);
+    }
 
     __host__ __device__ void init(long long seqs_, long long n_groups_, int r, int wg_,
                                   int wr_, long long warps_)
@@ -178,11 +220,12 @@ struct Split {
         warps = warps_;
     }
     __host__ __device__ long long n_items() const { return n_groups + n_res_items; }
-    __host__ __device__ long long lo(long long w) const { return floor_div(w * Tot, warps); }
+    __host__ __device__ long long lo(long long w) const { return div_floor(w * Tot, mW); }
     __host__ __device__ long long owner(long long pos) const
     {
-        return floor_div((pos + 1) * warps - 1, Tot);
+        return div_floor((pos + 1) * warps - 1, mT);
     }
+    __host__ __device__ long long seq_of(long long pos) const { return div_floor(pos, mC); }
     __host__ __device__ long long item_start(long long idx) const
     {
         return idx < n_groups ? idx * wg : n_groups * wg + (idx - n_groups) * wr;
@@ -192,9 +235,9 @@ struct Split {
     __host__ __device__ long long first_item_at(long long rel) const
     {
         long long gend = n_groups * wg;
-        if (n_groups > 0 && rel <= gend - wg) return floor_div(rel + wg - 1, wg);
+        if (n_groups > 0 && rel <= gend - wg) return div_floor(rel + wg - 1, mG);
         if (rel <= gend) return n_groups;
-        long long idx = n_groups + floor_div(rel - gend + wr - 1, wr);
+        long long idx = n_groups + div_floor(rel - gend + wr - 1, mR);
         return idx < n_items() ? idx : n_items();
     }
     // Items of sequence s owned by warp w: [*i0, *i1).

@@ -279,8 +279,13 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     // the last; the sequences between are whole.  Item indices fit 32 bits.
     Split sp;
     sp.init(p.seqs, p.n_groups, p.r, p.wg, p.wr, p.warps);
+    sp.mC = p.div_C;
+    sp.mT = p.div_Tot;
+    sp.mW = p.div_warps;
+    sp.mG = p.div_wg;
+    sp.mR = p.div_wr;
     const long long lo = sp.lo(gw), hi = sp.lo(gw + 1);
-    const int s_first = (int)floor_div(lo, sp.C), s_last = (int)floor_div(hi - 1, sp.C);
+    const int s_first = (int)sp.seq_of(lo), s_last = (int)sp.seq_of(hi - 1);
     const int n_items = (int)sp.n_items(), n_groups = (int)p.n_groups;
     int i_first, i_end;
     {
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     constexpr int QW = HG * D / 64;
     uint32_t qnext[QW];
     auto load_q = [&](int s) {
-        const int b = s / p.H_kv, hk = s - b * p.H_kv;
+        const int b = (int)div_floor(s, p.div_Hkv), hk = s - b * p.H_kv;
         const uint32_t *qg = (const uint32_t *)(p.q + ((long long)b * p.H_q + (long long)hk * HG) * D);
 #pragma unroll
         for (int i = 0; i < QW; ++i) qnext[i] = __ldg(qg + lane + 32 * i);
@@ -378,7 +383,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     for (int s = s_first; s <= s_last && !failed; ++s) {
         int i0, i1;
         seq_items(s, &i0, &i1);
-        const int b = s / p.H_kv, hk = s - b * p.H_kv;
+        const int b = (int)div_floor(s, p.div_Hkv), hk = s - b * p.H_kv;
 
         // Scaled query in shared memory (fp32) and the lane's q' inputs; then
         // the next sequence's query is requested (with four or more query

@@ -5,6 +5,9 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "kivi.h"
+#include "kivi_common.cuh"
+
 namespace kivi {
 
 // Quantize whole groups of 32 tokens into the packed store (prefill and the
@@ -42,6 +45,7 @@ struct DecodeParams {
     long long n_q;       // absolute position of residual slot 0
     int wg, wr;          // split weights of a group / a residual item
     long long warps;     // total warps of the split (<= total weight)
+    Magic div_C, div_Tot, div_warps, div_wg, div_wr, div_Hkv;   // divisions of the split
     int slots;           // partial slots per sequence
     float qscale;        // log2(e) / sqrt(D)
     uint32_t magic;      // bits of 2^23 (the code-to-float exponent)
@@ -58,5 +62,11 @@ cudaError_t launch_append(int D, const uint16_t *k, const uint16_t *v, uint16_t 
 int decode_warps_per_cta(int D, int HG, int pre_rope);
 cudaError_t launch_decode(int D, int HG, int dtype, int pre_rope, const DecodeParams &p,
                           cudaStream_t st);
+// Launch parameters of a decode call on cache c, validated as every decode
+// entry point validates them; the scratch pointers (partials, tickets) are
+// left null and `slots` is the least the split needs.
+kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q, float *out,
+                                           DecodeParams *p, int *D, int *HG, int *dtype,
+                                           int *pre_rope);
 
 }  // namespace kivi

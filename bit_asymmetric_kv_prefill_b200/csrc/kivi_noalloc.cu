@@ -19,12 +19,6 @@
 #include "kivi_common.cuh"
 #include "kivi_internal.h"
 
-namespace kivi {
-kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q, float *out,
-                                           DecodeParams *p, int *D, int *HG, int *dtype,
-                                           int *pre_rope);
-}
-
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device

@@ -5,6 +5,7 @@ import ctypes
 import itertools
 import subprocess
 
+import numpy as np
 import pytest
 
 import bit_asymmetric_kv_prefill_b200 as kivi
@@ -106,3 +107,51 @@ def test_decode_split_balances_weight():
         load[w] += sum(wg if i < n_groups else wr for i in range(i0, i1))
     per_seq = n_groups * wg + -(-r // 6) * wr
     assert sum(load) == per_seq * len(range(0, seqs, 17))
+
+
+def _split_reference(seqs, n_groups, r, wg, wr, warps, s, w):
+    """The split's definition in exact Python integers."""
+    n_res = -(-r // 6)
+    n_items = n_groups + n_res
+    C = n_groups * wg + n_res * wr
+    Tot = C * seqs
+
+    def lo(x):
+        return x * Tot // warps
+
+    def owner(pos):
+        return ((pos + 1) * warps - 1) // Tot
+
+    def first_item_at(rel):
+        gend = n_groups * wg
+        if n_groups > 0 and rel <= gend - wg:
+            return -(-rel // wg)
+        if rel <= gend:
+            return n_groups
+        return min(n_groups + -(-(rel - gend) // wr), n_items)
+
+    base = s * C
+    ra, rb = max(lo(w) - base, 0), min(lo(w + 1) - base, C)
+    i0 = i1 = 0
+    if ra < rb:
+        i0, i1 = first_item_at(ra), first_item_at(rb)
+        i1 = max(i1, i0)
+    return owner(base), owner(base + C - 1), i0, i1
+
+
+def test_decode_split_matches_exact_integer_definition():
+    """The split runs its divisions as reciprocal multiplies with a one-step
+    integer fix-up; on large shapes it must equal exact integer division."""
+    rng = np.random.default_rng(5)
+    for _ in range(60):
+        seqs = int(rng.integers(1, 4097))
+        n_groups = int(rng.integers(0, 1 << 20))
+        r = int(rng.integers(1, 129))
+        wg, wr = int(rng.integers(1, 17)), int(rng.integers(1, 17))
+        total = seqs * (n_groups * wg + -(-r // 6) * wr)
+        warps = min(int(rng.integers(1, 4737)), total)
+        for _ in range(20):
+            s, w = int(rng.integers(0, seqs)), int(rng.integers(0, warps))
+            got = tuple(kivi.decode_split(seqs, n_groups, r, wg, wr, warps, s, w))
+            assert got == _split_reference(seqs, n_groups, r, wg, wr, warps, s, w), \
+                (seqs, n_groups, r, wg, wr, warps, s, w)
