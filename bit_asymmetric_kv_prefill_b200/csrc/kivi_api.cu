@@ -41,6 +41,7 @@ kivi_status check_config(const kivi_config *c)
     if (c->G != kG) return KIVI_ERR_UNSUPPORTED;
     if (c->D != 64 && c->D != 128) return KIVI_ERR_UNSUPPORTED;
     if (c->pre_rope && !(c->rope_theta > 1.0f)) return KIVI_ERR_ARG;
+    if (c->pre_rope && c->T_max > kRopeMaxTokens) return KIVI_ERR_UNSUPPORTED;
     return KIVI_OK;
 }
 
@@ -468,10 +469,9 @@ extern "C" kivi_status kivi_decode_split(long long seqs, long long n_groups, int
     sp.set_magics();
     out[0] = sp.owner(seq * sp.C);
     out[1] = sp.owner((seq + 1) * sp.C - 1);
-    long long i0, i1;
-    sp.items(seq, warp, &i0, &i1);
-    out[2] = i0;
-    out[3] = i1;
+    const ItemRange it = sp.items(seq, warp);
+    out[2] = it.first;
+    out[3] = it.second;
     return KIVI_OK;
 }
 

@@ -11,6 +11,9 @@ namespace kivi {
 constexpr int kG = 32;          // tokens per key group, channels per value group
 constexpr int kResTok = 6;      // residual tokens per decode item (one stage)
 constexpr int kErrWaitTimeout = 1;
+// Longest pre-RoPE cache: decode reduces RoPE angles (position * inv_freq,
+// inv_freq <= 1) modulo 2pi exactly below 2^17 * 2pi = 823,549.
+constexpr long long kRopeMaxTokens = 823000;
 
 // ---------------------------------------------------------------------------
 // Packed group block.  One block per (sequence, group of 32 quantized tokens),
@@ -186,10 +189,14 @@ __host__ __device__ __forceinline__ unsigned long long mulhi64(unsigned long lon
 }
 
 // floor(a / d) for 0 <= a < 2^53, m = make_magic(d).
-__host__ __device__ __forceinline__ long long div_floor(long long a, const Magic &m)
+__host__ __device__ __forceinline__ long long div_floor(long long a, Magic m)
 {
     return (long long)(mulhi64((unsigned long long)a << m.sa, m.M) >> m.sb);
 }
+
+struct ItemRange {
+    long long first, second;
+};
 
 struct Split {
     long long seqs, n_groups, n_res_items, C, Tot, warps;
@@ -207,7 +214,7 @@ struct Split {
         mR = make_magic((unsigned long long)wr);
     }
 
-    __host__ __device__ void init(long long seqs_, long long n_groups_, int r, int wg_,
+    __host__ __device__ __forceinline__ void init(long long seqs_, long long n_groups_, int r, int wg_,
                                   int wr_, long long warps_)
     {
         seqs = seqs_;
@@ -219,20 +226,20 @@ struct Split {
         Tot = C * seqs;
         warps = warps_;
     }
-    __host__ __device__ long long n_items() const { return n_groups + n_res_items; }
-    __host__ __device__ long long lo(long long w) const { return div_floor(w * Tot, mW); }
-    __host__ __device__ long long owner(long long pos) const
+    __host__ __device__ __forceinline__ long long n_items() const { return n_groups + n_res_items; }
+    __host__ __device__ __forceinline__ long long lo(long long w) const { return div_floor(w * Tot, mW); }
+    __host__ __device__ __forceinline__ long long owner(long long pos) const
     {
         return div_floor((pos + 1) * warps - 1, mT);
     }
-    __host__ __device__ long long seq_of(long long pos) const { return div_floor(pos, mC); }
-    __host__ __device__ long long item_start(long long idx) const
+    __host__ __device__ __forceinline__ long long seq_of(long long pos) const { return div_floor(pos, mC); }
+    __host__ __device__ __forceinline__ long long item_start(long long idx) const
     {
         return idx < n_groups ? idx * wg : n_groups * wg + (idx - n_groups) * wr;
     }
     // Smallest item index whose start is >= rel (rel in [0, C]); n_items() if
     // there is none.
-    __host__ __device__ long long first_item_at(long long rel) const
+    __host__ __device__ __forceinline__ long long first_item_at(long long rel) const
     {
         long long gend = n_groups * wg;
         if (n_groups > 0 && rel <= gend - wg) return div_floor(rel + wg - 1, mG);
@@ -240,20 +247,16 @@ struct Split {
         long long idx = n_groups + div_floor(rel - gend + wr - 1, mR);
         return idx < n_items() ? idx : n_items();
     }
-    // Items of sequence s owned by warp w: [*i0, *i1).
-    __host__ __device__ void items(long long s, long long w, long long *i0, long long *i1) const
+    // Items of sequence s owned by warp w: [first, second).
+    __host__ __device__ __forceinline__ ItemRange items(long long s, long long w) const
     {
-        long long base = s * C;
-        long long a = lo(w), b = lo(w + 1);
-        long long ra = a > base ? a - base : 0;
-        long long rb = b < base + C ? b - base : C;
-        if (ra >= rb) {
-            *i0 = *i1 = 0;
-            return;
-        }
-        *i0 = first_item_at(ra);
-        *i1 = first_item_at(rb);
-        if (*i1 < *i0) *i1 = *i0;
+        const long long base = s * C;
+        const long long a = lo(w), b = lo(w + 1);
+        const long long ra = a > base ? a - base : 0;
+        const long long rb = b < base + C ? b - base : C;
+        if (ra >= rb) return ItemRange{0, 0};
+        const long long i0 = first_item_at(ra), i1 = first_item_at(rb);
+        return ItemRange{i0, i1 < i0 ? i0 : i1};
     }
 };
 

@@ -203,6 +203,25 @@ __device__ __forceinline__ float hfma_f32(uint32_t a, uint32_t b, float c)
 constexpr int kVTargetExp = 6;
 constexpr float kVLimit = 32768.0f;
 
+// RoPE angles.  (sin a, cos a) of an fp32 angle 0 <= a < 2^17 * 2pi: a is
+// reduced modulo 2pi by the method of Cody and Waite ("Software Manual for the
+// Elementary Functions", 1980) with 2pi split in four parts, P1 = 101/16,
+// P2 = -15/512 and P3 = -75/2^22 of at most 7 significant bits (each k*P_i
+// exact in fp32 for k = rint(a/2pi) < 2^17, and each partial difference
+// exact) and P4 = fl(2pi - P1 - P2 - P3).  The reduced angle is within 2^-22
+// of the exact one; the hardware sine and cosine of it add at most 2^-21.4.
+// Positions are limited accordingly when a pre-RoPE cache is created.
+__device__ __forceinline__ void rope_sincos(float a, float *sn, float *cn)
+{
+    const float k = __fadd_rn(__fmaf_rn(a, 0.15915494f, 12582912.0f), -12582912.0f);
+    float r = __fmaf_rn(-k, 6.3125f, a);
+    r = __fmaf_rn(-k, -0.029296875f, r);
+    r = __fmaf_rn(-k, __uint_as_float(0xb7960000u), r);
+    r = __fmaf_rn(-k, __uint_as_float(0x338885a3u), r);
+    *sn = __sinf(r);
+    *cn = __cosf(r);
+}
+
 template <int DT>
 __device__ __forceinline__ float to_f(uint16_t b)
 {
@@ -234,8 +253,13 @@ struct WarpSmem {
     static constexpr int QP = kStages * L::GB;      // float [HG][4][QPS]
     static constexpr int PP = QP + HG * 4 * QPS * 4;          // f16 [HG][NJ][PPS]
     static constexpr int QS = PP + HG * L::NJ * PPS * 2;      // float [HG][D]
-    static constexpr int SZ = QS + HG * D * 4;                // float2 [4][D/4] (RoPE)
-    static constexpr int BAR = SZ + (ROPE ? D * 8 : 0);       // uint64 [kStages]
+    static constexpr int SZS = D / 4 + 4;                     // padded slice row (float2)
+    static constexpr int SZ = QS + HG * D * 4;                // float2 [4][SZS] (RoPE)
+    static constexpr int QRS = D / 8 + 2;                     // padded pair row (float2)
+    static constexpr int QR = SZ + (ROPE ? 4 * SZS * 8 : 0);  // float2 [HG][4][QRS] (RoPE)
+    static constexpr int FRS = D / 8 + 4;                     // padded frequency row (float)
+    static constexpr int FR = QR + (ROPE ? HG * 4 * QRS * 8 : 0);    // float [4][FRS] (RoPE)
+    static constexpr int BAR = FR + (ROPE ? 4 * FRS * 4 : 0);        // uint64 [kStages]
     static constexpr int BYTES = (BAR + kStages * 8 + 15) / 16 * 16;
 };
 
@@ -270,6 +294,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     uint16_t *pp = (uint16_t *)(ws + W::PP);
     float *qs = (float *)(ws + W::QS);
     float2 *sz = (float2 *)(ws + W::SZ);
+    float2 *qr = (float2 *)(ws + W::QR);
+    float *frq = (float *)(ws + W::FR);
     const uint32_t bar0 = smem_addr(ws + W::BAR);
     const uint32_t magic = p.magic;
     const float2 neg = make_float2(p.neg_magic, p.neg_magic);
@@ -284,17 +310,16 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     sp.mW = p.div_warps;
     sp.mG = p.div_wg;
     sp.mR = p.div_wr;
-    const long long lo = sp.lo(gw), hi = sp.lo(gw + 1);
+    // (The warp index enters as an opaque register: measured, this keeps the
+    // split's 64-bit arithmetic on the vector pipes and the prologue short.)
+    long long gwo = gw;
+    asm volatile("" : "+l"(gwo));
+    const long long lo = sp.lo(gwo), hi = sp.lo(gwo + 1);
     const int s_first = (int)sp.seq_of(lo), s_last = (int)sp.seq_of(hi - 1);
     const int n_items = (int)sp.n_items(), n_groups = (int)p.n_groups;
     int i_first, i_end;
-    {
-        long long a0, a1, b0, b1;
-        sp.items(s_first, gw, &a0, &a1);
-        sp.items(s_last, gw, &b0, &b1);
-        i_first = (int)a0;
-        i_end = (int)b1;
-    }
+    i_first = (int)sp.items(s_first, gwo).first;
+    i_end = (int)sp.items(s_last, gwo).second;
     auto seq_items = [&](int s, int *i0, int *i1) {
         *i0 = s == s_first ? i_first : 0;
         *i1 = s == s_last ? i_end : n_items;
@@ -380,6 +405,13 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     // at, 2^-(2*((t mod TPW)*CPL/2 mod 4)).
     const float vtok = pow2i(-2 * (((lane % TPW) * (CPL / 2)) & 3));
 
+    // RoPE: inverse frequencies of the pairs of slice c4, frq[c4][i] for pair
+    // c4*D/8 + i (rows padded against bank conflicts).
+    if constexpr (ROPE) {
+        for (int e = lane; e < D / 2; e += 32) frq[(e / HALF) * W::FRS + e % HALF] = __ldg(p.inv_freq + e);
+        __syncwarp();
+    }
+
     for (int s = s_first; s <= s_last && !failed; ++s) {
         int i0, i1;
         seq_items(s, &i0, &i1);
@@ -397,6 +429,16 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
             qs[e + 1] = to_f<DT>((uint16_t)(qnext[i] >> 16)) * p.qscale;
         }
         __syncwarp();
+        if constexpr (ROPE) {
+            // Rotate-half partners side by side: qr[h][cs][i] = (q_i, q_{i+D/2})
+            // of slice cs, channel i = cs*D/8 + i'.
+            for (int e = lane; e < HG * 4 * HALF; e += 32) {
+                const int h = e / (4 * HALF), r = e % (4 * HALF), c4 = r / HALF, i = r % HALF;
+                qr[(h * 4 + c4) * W::QRS + i] =
+                    make_float2(qs[h * D + c4 * HALF + i], qs[h * D + D / 2 + c4 * HALF + i]);
+            }
+            __syncwarp();
+        }
         if (HG <= 2 && s < s_last) load_q(s + 1);
         float qreg[HG][QPL], qsc[HG][QPL];
 #pragma unroll
@@ -485,7 +527,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     // Scales carry the inverse of each code pair's shift.
 #pragma unroll
                     for (int e = 0; e < QPL; ++e)
-                        sz[pcs * (D / 4) + pL0 + e] =
+                        sz[pcs * W::SZS + pL0 + e] =
                             make_float2(f16f(km[e]) * pair_scale(((pL0 + e) & 15) >> 1), f16f(km[QPL + e]));
                 }
                 __syncwarp();
@@ -538,42 +580,54 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
 #pragma unroll
                         for (int h = 0; h < HG; ++h) part[t][h] = acc[t][h].x + acc[t][h].y;
                 } else {
-                    // Dequantize, rotate at absolute positions, dot with q.
+                    // Dequantize, rotate at absolute positions, dot with q, two
+                    // rotate-half pairs (i, i+1) of the slice at a time.
                     const long long tbase = (long long)it * kG + 4 * tq;
 #pragma unroll 1
                     for (int t = 0; t < 4; ++t) {
-                        float kh[D / 4];
-#pragma unroll
-                        for (int k = 0; k < KW; ++k) {
-                            const uint32_t w = kw[t * KW + k], w16 = w >> 16;
-#pragma unroll
-                            for (int i = 0; i < 16; i += 2) {
-                                const float2 c = code_pair(w, w16, i / 2, magic, neg);
-                                const float2 s0 = sz[cs * (D / 4) + 16 * k + i];
-                                const float2 s1 = sz[cs * (D / 4) + 16 * k + i + 1];
-                                kh[16 * k + i] = fmaf(c.x, s0.x, s0.y);
-                                kh[16 * k + i + 1] = fmaf(c.y, s1.x, s1.y);
-                            }
-                        }
                         const float pos = (float)(tbase + t);
+                        // Token t's words, picked by selects (an index by the
+                        // rolled t would move kw to the stack).
+                        uint32_t wt[KW];
 #pragma unroll
-                        for (int i = 0; i < HALF; ++i) {
-                            const float a = __fmul_rn(pos, __ldg(p.inv_freq + cs * HALF + i));
-                            float sn, cn;
-                            sincosf(a, &sn, &cn);
-                            const float x = kh[i], y = kh[HALF + i];
-                            kh[i] = x * cn - y * sn;
-                            kh[HALF + i] = y * cn + x * sn;
+                        for (int k = 0; k < KW; ++k)
+                            wt[k] = t == 0 ? kw[k] : t == 1 ? kw[KW + k] : t == 2 ? kw[2 * KW + k] : kw[3 * KW + k];
+                        float d0[HG], d1[HG];
+#pragma unroll
+                        for (int h = 0; h < HG; ++h) d0[h] = d1[h] = 0.f;
+#pragma unroll 2
+                        for (int i = 0; i < HALF; i += 2) {
+                            // Local channels i, i+1 (first RoPE half) and HALF+i,
+                            // HALF+i+1 (their partners); word k = L/16, pair (L%16)/2.
+                            const int Lx = i, Ly = HALF + i;
+                            const uint32_t wx = wt[Lx / 16], wy = wt[Ly / 16];
+                            const float2 cx = code_pair(wx, wx >> 16, (Lx % 16) / 2, magic, neg);
+                            const float2 cy = code_pair(wy, wy >> 16, (Ly % 16) / 2, magic, neg);
+                            const float2 sx0 = sz[cs * W::SZS + Lx], sx1 = sz[cs * W::SZS + Lx + 1];
+                            const float2 sy0 = sz[cs * W::SZS + Ly], sy1 = sz[cs * W::SZS + Ly + 1];
+                            const float x0 = fmaf(cx.x, sx0.x, sx0.y), x1 = fmaf(cx.y, sx1.x, sx1.y);
+                            const float y0 = fmaf(cy.x, sy0.x, sy0.y), y1 = fmaf(cy.y, sy1.x, sy1.y);
+                            const float2 f2 = *(const float2 *)(frq + cs * W::FRS + i);
+                            float sn0, cn0, sn1, cn1;
+                            rope_sincos(__fmul_rn(pos, f2.x), &sn0, &cn0);
+                            rope_sincos(__fmul_rn(pos, f2.y), &sn1, &cn1);
+                            const float rx0 = x0 * cn0 - y0 * sn0, ry0 = y0 * cn0 + x0 * sn0;
+                            const float rx1 = x1 * cn1 - y1 * sn1, ry1 = y1 * cn1 + x1 * sn1;
+#pragma unroll
+                            for (int h = 0; h < HG; ++h) {
+                                const float4 qq = *(const float4 *)(qr + (h * 4 + cs) * W::QRS + i);
+                                d0[h] = fmaf(qq.x, rx0, d0[h]);
+                                d1[h] = fmaf(qq.y, ry0, d1[h]);
+                                d0[h] = fmaf(qq.z, rx1, d0[h]);
+                                d1[h] = fmaf(qq.w, ry1, d1[h]);
+                            }
                         }
 #pragma unroll
                         for (int h = 0; h < HG; ++h) {
-                            float d0 = 0.f, d1 = 0.f;
+                            const float d = d0[h] + d1[h];
 #pragma unroll
-                            for (int i = 0; i < HALF; ++i) {
-                                d0 = fmaf(qs[h * D + cs * HALF + i], kh[i], d0);
-                                d1 = fmaf(qs[h * D + D / 2 + cs * HALF + i], kh[HALF + i], d1);
-                            }
-                            part[t][h] = d0 + d1;
+                            for (int u = 0; u < 4; ++u)
+                                if (u == t) part[u][h] = d;
                         }
                     }
                 }
@@ -710,9 +764,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                             const float pos = (float)(p.n_q + t0 + tq);
 #pragma unroll
                             for (int i = 0; i < HALF; ++i) {
-                                const float a = __fmul_rn(pos, __ldg(p.inv_freq + cs * HALF + i));
                                 float sn, cn;
-                                sincosf(a, &sn, &cn);
+                                rope_sincos(__fmul_rn(pos, frq[cs * W::FRS + i]), &sn, &cn);
                                 const float x = kx[0][i], y = kx[1][i];
                                 kx[0][i] = x * cn - y * sn;
                                 kx[1][i] = y * cn + x * sn;
@@ -778,12 +831,19 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         const long long last = sp.owner(((long long)s + 1) * sp.C - 1);
         const int count = (int)(last - first + 1);
         const int slot = (int)(gw - first);
-        float lt[HG], zt[HG][NJ];
+        // lt: the softmax sum; zt: the zero term of the lane's value group jl
+        // (picked by selects: a lane-dependent index would put the array on
+        // the stack).
+        float lt[HG], zt[HG];
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
             lt[h] = warp_sum(lsum[h]);
+            zt[h] = 0.f;
 #pragma unroll
-            for (int j = 0; j < NJ; ++j) zt[h][j] = warp_sum(zacc[h][j]);
+            for (int j = 0; j < NJ; ++j) {
+                const float zj = warp_sum(zacc[h][j]);
+                zt[h] = jl == j ? zj : zt[h];
+            }
         }
         // Undo the per-pair factor 2^(2m), join the two token halves and add
         // the zero term: lane (vco, vth) then holds channels vco*CPL + c.
@@ -796,8 +856,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 const float f = pow2i(24 - c - ev[h]);   // 2^(24 - 2mm - ev)
                 const float x = a.x + __shfl_xor_sync(FULL, a.x, 16);
                 const float y = a.y + __shfl_xor_sync(FULL, a.y, 16);
-                o[h][c] = fmaf(x, f, zt[h][jl]);
-                o[h][c + 1] = fmaf(y, f, zt[h][jl]);
+                o[h][c] = fmaf(x, f, zt[h]);
+                o[h][c + 1] = fmaf(y, f, zt[h]);
             }
         float *outrow = p.out + ((long long)b * p.H_q + (long long)hk * HG) * D;
         if (count == 1) {
@@ -833,41 +893,53 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         is_last = __shfl_sync(FULL, is_last, 0);
         if (!is_last) continue;
         __threadfence();
-        // Log-sum-exp merge of the `count` partials of sequence s: lanes load
-        // the (m, l) of 32 partials at a time, then every lane streams its
-        // channels of all partials with independent loads.
+        // Log-sum-exp merge of the `count` partials of sequence s in one pass:
+        // each round trip loads (m, l) and the lane's channels of 8 partials
+        // together and folds them into a running (max, sum, row).
 #pragma unroll 1
         for (int h = 0; h < HG; ++h) {
-            float mx = -INFINITY;
-            for (int k = lane; k < count; k += 32)
-                mx = fmaxf(mx, __ldcg(pbase + ((long long)k * HG + h) * PSTRIDE + D));
-            mx = warp_max(mx);
-            float lacc = 0.f;
+            float M = -INFINITY, lacc = 0.f;
             float oo[QPL];
 #pragma unroll
             for (int c = 0; c < QPL; ++c) oo[c] = 0.f;
-            for (int k0 = 0; k0 < count; k0 += 32) {
-                const int kk = k0 + lane;
-                float wk = 0.f;
-                if (kk < count) {
-                    const float2 ml = __ldcg((const float2 *)(pbase + ((long long)kk * HG + h) * PSTRIDE + D));
-                    wk = ex2(ml.x - mx);
-                    lacc = fmaf(wk, ml.y, lacc);
-                }
-                const int n = min(32, count - k0);
-#pragma unroll 8
-                for (int j = 0; j < n; ++j) {
-                    const float wj = __shfl_sync(FULL, wk, j);
-                    const float *pk = pbase + ((long long)(k0 + j) * HG + h) * PSTRIDE + lane * QPL;
+            for (int k0 = 0; k0 < count; k0 += 8) {
+                float2 ml[8];
+                float v[8][QPL];
 #pragma unroll
-                    for (int c = 0; c < QPL; c += 2) {
-                        const float2 v = __ldcg((const float2 *)(pk + c));
-                        oo[c] = fmaf(wj, v.x, oo[c]);
-                        oo[c + 1] = fmaf(wj, v.y, oo[c + 1]);
+                for (int j = 0; j < 8; ++j) {
+                    if (k0 + j < count) {
+                        const float *row = pbase + ((long long)(k0 + j) * HG + h) * PSTRIDE;
+                        ml[j] = __ldcg((const float2 *)(row + D));
+#pragma unroll
+                        for (int c = 0; c < QPL; c += 2) {
+                            const float2 x = __ldcg((const float2 *)(row + lane * QPL + c));
+                            v[j][c] = x.x;
+                            v[j][c + 1] = x.y;
+                        }
+                    } else {
+                        ml[j] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+                        for (int c = 0; c < QPL; ++c) v[j][c] = 0.f;
                     }
                 }
+                float mx = M;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mx = fmaxf(mx, ml[j].x);
+                if (mx == -INFINITY) continue;   // only empty partials so far
+                const float a = ex2(M - mx);
+                lacc *= a;
+#pragma unroll
+                for (int c = 0; c < QPL; ++c) oo[c] *= a;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float wj = ex2(ml[j].x - mx);
+                    lacc = fmaf(wj, ml[j].y, lacc);
+#pragma unroll
+                    for (int c = 0; c < QPL; ++c) oo[c] = fmaf(wj, v[j][c], oo[c]);
+                }
+                M = mx;
             }
-            const float inv = 1.0f / warp_sum(lacc);
+            const float inv = 1.0f / lacc;
 #pragma unroll
             for (int c = 0; c < QPL; c += 2)
                 *(float2 *)(outrow + h * D + lane * QPL + c) = make_float2(oo[c] * inv, oo[c + 1] * inv);

@@ -399,17 +399,18 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quant_kernel(QuantParams p)
 }
 
 // Plain append: token rows [seqs][D] -> residual slot `slot` of each sequence.
+// One 16-byte chunk of k_t and of v_t per thread; N16 = D/8 chunks per row.
+template <int N16>
 __global__ void append_kernel(const uint4 *k, const uint4 *v, uint4 *resK, uint4 *resV,
-                              long long seqs, int R, int slot, int n16)
+                              long long seqs, int R, int slot)
 {
-    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    long long total = seqs * n16;
-    if (i >= total) return;
-    long long s = i / n16;
-    int c = (int)(i % n16);
-    long long d = (s * R + slot) * n16 + c;
-    resK[d] = k[i];
-    resV[d] = v[i];
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= seqs * N16) return;
+    const long long s = i / N16;
+    const long long d = (s * R + slot) * N16 + (i % N16);
+    const uint4 a = __ldcs(k + i), b = __ldcs(v + i);
+    resK[d] = a;
+    resV[d] = b;
 }
 
 int num_sms()
@@ -451,13 +452,15 @@ cudaError_t launch_quant(int D, int dtype, const QuantParams &p, cudaStream_t st
 cudaError_t launch_append(int D, const uint16_t *k, const uint16_t *v, uint16_t *resK,
                           uint16_t *resV, long long seqs, int R, int slot, cudaStream_t st)
 {
-    const int n16 = D / 8;
-    const long long total = seqs * n16;
-    const int block = 256;
+    const long long total = seqs * (D / 8);
+    const int block = 128;
     const long long grid = (total + block - 1) / block;
-    append_kernel<<<(unsigned)grid, block, 0, st>>>((const uint4 *)k, (const uint4 *)v,
-                                                     (uint4 *)resK, (uint4 *)resV, seqs, R, slot,
-                                                     n16);
+    if (D == 64)
+        append_kernel<8><<<(unsigned)grid, block, 0, st>>>((const uint4 *)k, (const uint4 *)v,
+                                                          (uint4 *)resK, (uint4 *)resV, seqs, R, slot);
+    else
+        append_kernel<16><<<(unsigned)grid, block, 0, st>>>((const uint4 *)k, (const uint4 *)v,
+                                                           (uint4 *)resK, (uint4 *)resV, seqs, R, slot);
     return cudaGetLastError();
 }
 

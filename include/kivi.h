@@ -76,7 +76,9 @@ typedef enum {
  * Cache geometry.  Supported: D in {64, 128}, G == 32, R a positive multiple
  * of G, dtype KIVI_F16 or KIVI_BF16, 1 <= T_max.  T_max bounds the total
  * number of tokens (prefill plus appends).  pre_rope != 0 stores keys before
- * RoPE and rotates them in decode with base rope_theta (e.g. 10000).
+ * RoPE and rotates them in decode with base rope_theta (e.g. 10000); such a
+ * cache supports T_max <= 823000 (the decode's angle reduction is exact for
+ * angles below 2^17 * 2pi), larger T_max gives KIVI_ERR_UNSUPPORTED.
  * workspace: optional caller-owned device memory of at least
  * kivi_cache_required_bytes(cfg) bytes, 256-byte aligned, which then holds
  * every device buffer of the cache (the library allocates nothing); it must
