@@ -236,6 +236,44 @@ __device__ __forceinline__ float warp_sum(float x)
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
     return x;
 }
+// Reduce-scatter of N per-lane values: at each level (lane offset OFF, OFF/2,
+// ...) a lane keeps half of its values and adds its partner's copy of them,
+// until one value is left, that of index h = the lane's bits OFF, OFF/2, ...
+// (most significant first), summed over those lanes.
+template <int N, int OFF>
+__device__ __forceinline__ float reduce_scatter(const float (&v)[N], int lane)
+{
+    if constexpr (N == 1) {
+        return v[0];
+    } else {
+        const bool up = lane & OFF;
+        float nv[N / 2];
+#pragma unroll
+        for (int i = 0; i < N / 2; ++i) {
+            const float keep = up ? v[N / 2 + i] : v[i];
+            const float send = up ? v[i] : v[N / 2 + i];
+            nv[i] = keep + __shfl_xor_sync(FULL, send, OFF);
+        }
+        return reduce_scatter<N / 2, OFF / 2>(nv, lane);
+    }
+}
+// out[h] = sum over the warp of v[h], for every h, in every lane (N a power
+// of two up to 16): a reduce-scatter, the rest of the butterfly, a gather.
+template <int N>
+__device__ __forceinline__ void warp_sum_n(const float (&v)[N], float (&out)[N], int lane)
+{
+    if constexpr (N == 1) {
+        out[0] = warp_sum(v[0]);
+    } else {
+        constexpr int LOG = N == 2 ? 1 : N == 4 ? 2 : N == 8 ? 3 : 4;
+        float x = reduce_scatter<N, 16>(v, lane);
+#pragma unroll
+        for (int o = 16 >> LOG; o > 0; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
+#pragma unroll
+        for (int h = 0; h < N; ++h) out[h] = __shfl_sync(FULL, x, h << (5 - LOG));
+    }
+}
+
 __device__ __forceinline__ float warp_max(float x)
 {
 #pragma unroll
@@ -248,11 +286,12 @@ template <int D, int HG, bool ROPE>
 struct WarpSmem {
     using L = Layout<D>;
     static constexpr int QPS = D / 4 + 4;           // padded q' slice (floats)
-    static constexpr int PPS = 40;                  // padded weight row (f16)
+    static constexpr int PPS = 40;                  // padded weight row (f16), one head
+    static constexpr int PPS2 = 36;                 // padded weight row (u32), head pairs
     static constexpr int RING = 0;                  // kStages x GB
     static constexpr int QP = kStages * L::GB;      // float [HG][4][QPS]
     static constexpr int PP = QP + HG * 4 * QPS * 4;          // f16 [HG][NJ][PPS]
-    static constexpr int QS = PP + HG * L::NJ * PPS * 2;      // float [HG][D]
+    static constexpr int QS = PP + (HG == 1 ? L::NJ * PPS * 2 : (HG / 2) * L::NJ * PPS2 * 4);  // float [HG][D]
     static constexpr int SZS = D / 4 + 4;                     // padded slice row (float2)
     static constexpr int SZ = QS + HG * D * 4;                // float2 [4][SZS] (RoPE)
     static constexpr int QRS = D / 8 + 2;                     // padded pair row (float2)
@@ -453,12 +492,12 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         float2 accV[HG][CPL / 2];
         // accV[h][mm] holds sum_t p_t s_t c_t 2^(2mm-24) * 2^ev[h].
         int ev[HG];
-        float evs[HG];   // 2^ev
+        float evs[HG];   // 2^ev * vtok
         bool ev_fresh[HG];
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
             ev[h] = 0;
-            evs[h] = 1.0f;
+            evs[h] = vtok;
             ev_fresh[h] = true;
             m[h] = -INFINITY;
             lsum[h] = 0.f;
@@ -509,20 +548,21 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                         sk[e] = f16f(km[e]);
                         zk[e] = f16f(km[QPL + e]);
                     }
+                    float bp[HG];
 #pragma unroll
                     for (int h = 0; h < HG; ++h) {
-                        float bp = 0.f;
+                        bp[h] = 0.f;
                         float qv[QPL];
 #pragma unroll
                         for (int e = 0; e < QPL; ++e) {
                             qv[e] = qsc[h][e] * sk[e];
-                            bp = fmaf(qreg[h][e], zk[e], bp);
+                            bp[h] = fmaf(qreg[h][e], zk[e], bp[h]);
                         }
                         float *dstq = qp + (h * 4 + pcs) * W::QPS + pL0;
 #pragma unroll
                         for (int e = 0; e < QPL; e += 2) *(float2 *)(dstq + e) = make_float2(qv[e], qv[e + 1]);
-                        bias[h] = warp_sum(bp);
                     }
+                    warp_sum_n<HG>(bp, bias, lane);
                 } else {
                     // Scales carry the inverse of each code pair's shift.
 #pragma unroll
@@ -603,10 +643,10 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                             const uint32_t wx = wt[Lx / 16], wy = wt[Ly / 16];
                             const float2 cx = code_pair(wx, wx >> 16, (Lx % 16) / 2, magic, neg);
                             const float2 cy = code_pair(wy, wy >> 16, (Ly % 16) / 2, magic, neg);
-                            const float2 sx0 = sz[cs * W::SZS + Lx], sx1 = sz[cs * W::SZS + Lx + 1];
-                            const float2 sy0 = sz[cs * W::SZS + Ly], sy1 = sz[cs * W::SZS + Ly + 1];
-                            const float x0 = fmaf(cx.x, sx0.x, sx0.y), x1 = fmaf(cx.y, sx1.x, sx1.y);
-                            const float y0 = fmaf(cy.x, sy0.x, sy0.y), y1 = fmaf(cy.y, sy1.x, sy1.y);
+                            const float4 sx = *(const float4 *)(sz + cs * W::SZS + Lx);
+                            const float4 sy = *(const float4 *)(sz + cs * W::SZS + Ly);
+                            const float x0 = fmaf(cx.x, sx.x, sx.y), x1 = fmaf(cx.y, sx.z, sx.w);
+                            const float y0 = fmaf(cy.x, sy.x, sy.y), y1 = fmaf(cy.y, sy.z, sy.w);
                             const float2 f2 = *(const float2 *)(frq + cs * W::FRS + i);
                             float sn0, cn0, sn1, cn1;
                             rope_sincos(__fmul_rn(pos, f2.x), &sn0, &cn0);
@@ -650,19 +690,22 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 softmax_step(sc, pr, true);
 
                 // Token weights b = p s 2^ev (times the lane's shift factor)
-                // for token `lane`, as f16 rows [h][j][token].
+                // for token `lane`, as f16 rows [h][j][token]; with two or
+                // more query heads, head pairs share a word: u32 rows
+                // [j][h/2][token] holding (b_h, b_h+1).
                 const uint16_t *vm = (const uint16_t *)(st + L::VM + lane * (D / 8));
                 float svj[NJ];
 #pragma unroll
                 for (int j = 0; j < NJ; ++j) {
-                    svj[j] = f16f(vm[j]) * vtok;
+                    svj[j] = f16f(vm[j]);
                     const float zvj = f16f(vm[NJ + j]);
 #pragma unroll
                     for (int h = 0; h < HG; ++h) zacc[h][j] = fmaf(pr[h], zvj, zacc[h][j]);
                 }
+                float fh[HG];
 #pragma unroll
                 for (int h = 0; h < HG; ++h) {
-                    float f = pr[h] * evs[h];
+                    float f = pr[h] * evs[h];   // evs carries the lane's vtok
                     float bm = 0.f;
 #pragma unroll
                     for (int j = 0; j < NJ; ++j) bm = fmaxf(bm, f * svj[j]);
@@ -683,15 +726,27 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                                 accV[h][c].x = accV[h][c].x * pow2i(d1) * pow2i(d2);
                                 accV[h][c].y = accV[h][c].y * pow2i(d1) * pow2i(d2);
                             }
-                            evs[h] = pow2i(en);
+                            evs[h] = pow2i(en) * vtok;
                             f = pr[h] * evs[h];
                             ev[h] = en;
                             ev_fresh[h] = false;
                         }
                     }
+                    fh[h] = f;
+                }
+                if constexpr (HG == 1) {
 #pragma unroll
                     for (int j = 0; j < NJ; ++j)
-                        pp[(h * NJ + j) * W::PPS + lane] = __half_as_ushort(__float2half_rn(f * svj[j]));
+                        pp[j * W::PPS + lane] = __half_as_ushort(__float2half_rn(fh[0] * svj[j]));
+                } else {
+                    uint32_t *pp32 = (uint32_t *)pp;
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j)
+#pragma unroll
+                        for (int hp = 0; hp < HG / 2; ++hp) {
+                            const __half2 b2 = __floats2half2_rn(fh[2 * hp] * svj[j], fh[2 * hp + 1] * svj[j]);
+                            pp32[(j * (HG / 2) + hp) * W::PPS2 + lane] = *(const uint32_t *)&b2;
+                        }
                 }
                 __syncwarp();
 
@@ -706,14 +761,23 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     vw[4 * c + 2] = v4.z;
                     vw[4 * c + 3] = v4.w;
                 }
-                // The 16 token weights of the lane's tokens, two per word.
-                uint32_t pb[HG][8];
+                // The weights of the lane's 16 tokens: one head, two tokens
+                // per word (HG == 1), or one token, two heads per word.
+                constexpr int PBW = HG == 1 ? 8 : 16;
+                uint32_t pb[HG == 1 ? 1 : HG / 2][PBW];
 #pragma unroll
-                for (int h = 0; h < HG; ++h) {
-                    const uint4 *src = (const uint4 *)(pp + (h * NJ + jl) * W::PPS + 16 * vth);
-                    const uint4 a = src[0], b = src[1];
-                    pb[h][0] = a.x; pb[h][1] = a.y; pb[h][2] = a.z; pb[h][3] = a.w;
-                    pb[h][4] = b.x; pb[h][5] = b.y; pb[h][6] = b.z; pb[h][7] = b.w;
+                for (int hp = 0; hp < (HG == 1 ? 1 : HG / 2); ++hp) {
+                    const uint4 *src = HG == 1
+                        ? (const uint4 *)(pp + jl * W::PPS + 16 * vth)
+                        : (const uint4 *)((const uint32_t *)pp + (jl * (HG / 2) + hp) * W::PPS2 + 16 * vth);
+#pragma unroll
+                    for (int c = 0; c < PBW / 4; ++c) {
+                        const uint4 a = src[c];
+                        pb[hp][4 * c] = a.x;
+                        pb[hp][4 * c + 1] = a.y;
+                        pb[hp][4 * c + 2] = a.z;
+                        pb[hp][4 * c + 3] = a.w;
+                    }
                 }
 #pragma unroll
                 for (int u = 0; u < L::WPL; ++u) {
@@ -726,8 +790,11 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                             const uint32_t x = (i < 4 ? w : w8) & (0x00030003u << (2 * (i & 3)));
 #pragma unroll
                             for (int h = 0; h < HG; ++h) {
-                                const uint32_t bw = pb[h][(u * TPW + tt) >> 1];
-                                if ((tt & 1) == 0) {
+                                // The weight's half: the token's parity (one
+                                // head) or the head's parity (head pairs).
+                                const uint32_t bw = HG == 1 ? pb[0][(u * TPW + tt) >> 1] : pb[h / 2][u * TPW + tt];
+                                const bool odd = HG == 1 ? (tt & 1) : (h & 1);
+                                if (!odd) {
                                     accV[h][mm].x = hfma_f32<0, 0>(x, bw, accV[h][mm].x);
                                     accV[h][mm].y = hfma_f32<1, 0>(x, bw, accV[h][mm].y);
                                 } else {
