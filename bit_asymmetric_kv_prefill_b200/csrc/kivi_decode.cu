@@ -53,7 +53,12 @@ namespace kivi {
 #endif
 
 constexpr unsigned FULL = 0xffffffffu;
-constexpr int kStages = KIVI_DECODE_STAGES;
+#ifndef KIVI_DECODE_STAGES_GQA
+#define KIVI_DECODE_STAGES_GQA 3   // four or more query heads per kv head
+#endif
+// Ring depth (shared-memory stages per warp) of an instantiation.
+template <int HG>
+constexpr int ring_stages() { return HG >= 4 ? KIVI_DECODE_STAGES_GQA : KIVI_DECODE_STAGES; }
 constexpr float kRescaleSlack = 8.0f;
 constexpr int kWaitLimit = 1 << 22;
 
@@ -288,8 +293,9 @@ struct WarpSmem {
     static constexpr int QPS = D / 4 + 4;           // padded q' slice (floats)
     static constexpr int PPS = 40;                  // padded weight row (f16), one head
     static constexpr int PPS2 = 36;                 // padded weight row (u32), head pairs
-    static constexpr int RING = 0;                  // kStages x GB
-    static constexpr int QP = kStages * L::GB;      // float [HG][4][QPS]
+    static constexpr int NST = ring_stages<HG>();
+    static constexpr int RING = 0;                  // NST x GB
+    static constexpr int QP = NST * L::GB;          // float [HG][4][QPS]
     static constexpr int PP = QP + HG * 4 * QPS * 4;          // f16 [HG][NJ][PPS]
     static constexpr int QS = PP + (HG == 1 ? L::NJ * PPS * 2 : (HG / 2) * L::NJ * PPS2 * 4);  // float [HG][D]
     static constexpr int SZS = D / 4 + 4;                     // padded slice row (float2)
@@ -298,8 +304,8 @@ struct WarpSmem {
     static constexpr int QR = SZ + (ROPE ? 4 * SZS * 8 : 0);  // float2 [HG][4][QRS] (RoPE)
     static constexpr int FRS = D / 8 + 4;                     // padded frequency row (float)
     static constexpr int FR = QR + (ROPE ? HG * 4 * QRS * 8 : 0);    // float [4][FRS] (RoPE)
-    static constexpr int BAR = FR + (ROPE ? 4 * FRS * 4 : 0);        // uint64 [kStages]
-    static constexpr int BYTES = (BAR + kStages * 8 + 15) / 16 * 16;
+    static constexpr int BAR = FR + (ROPE ? 4 * FRS * 4 : 0);        // uint64 [NST]
+    static constexpr int BYTES = (BAR + NST * 8 + 15) / 16 * 16;
 };
 
 template <int D, int HG, bool ROPE>
@@ -321,6 +327,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     constexpr int NW = DecodeShape<D, HG, ROPE>::NW;
     constexpr int CPL = L::CPL, QPL = L::QPL, NJ = L::NJ, KW = L::KW, HALF = L::HALF, TPW = L::TPW;
     constexpr int PSTRIDE = D + 4;
+    constexpr int kSt = W::NST;
 
     extern __shared__ __align__(128) unsigned char smem_all[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -338,6 +345,12 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     const uint32_t bar0 = smem_addr(ws + W::BAR);
     const uint32_t magic = p.magic;
     const float2 neg = make_float2(p.neg_magic, p.neg_magic);
+
+    // The ring's barriers first: they need nothing from the split.
+    if (lane == 0) {
+        for (int i = 0; i < kSt; ++i) mbar_init(bar0 + 8 * i, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
 
     // This warp's share of the flattened (sequence, item) list: sequences
     // s_first..s_last, items [i_first, ...) of the first and [..., i_end) of
@@ -375,12 +388,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
 #pragma unroll
         for (int i = 0; i < QW; ++i) qnext[i] = __ldg(qg + lane + 32 * i);
     };
-    load_q(s_first);
-
-    if (lane == 0) {
-        for (int i = 0; i < kStages; ++i) mbar_init(bar0 + 8 * i, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
+    load_q(s_first);   // ahead of the ring's copies, which it would queue behind
     __syncwarp();
 
     // Prefetch iterator over the warp's items, possibly across sequences.
@@ -403,7 +411,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         if (pf_i >= pf_e) return;
         const uint32_t bar = bar0 + 8 * ist;
         const uint32_t dst = ring_s + ist * L::GB;
-        ist = ist + 1 == kStages ? 0 : ist + 1;
+        ist = ist + 1 == kSt ? 0 : ist + 1;
         if (pf_i < n_groups) {
             const uint8_t *src = p.packed + ((long long)pf_s * p.ngcap + pf_i) * (long long)L::GB;
             lane0_expect_copy(lane, bar, dst, src, L::GB, L::GB);
@@ -418,7 +426,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         ++issued;
         ++pf_i;
     };
-    for (int i = 0; i < kStages; ++i) issue_next();
+    for (int i = 0; i < kSt; ++i) issue_next();
 
     bool failed = false;
     auto wait_stage = [&]() -> bool {
@@ -429,7 +437,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     };
     auto next_stage = [&]() {
         ++consumed;
-        if (++cst == kStages) {
+        if (++cst == kSt) {
             cst = 0;
             cph ^= 1u;
         }
@@ -479,6 +487,9 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
             __syncwarp();
         }
         if (HG <= 2 && s < s_last) load_q(s + 1);
+        // The q'-writer lane's query channels, plain and with their pair-shift
+        // factors folded in (held in registers: measured faster than re-reading
+        // shared memory every group, even with four heads).
         float qreg[HG][QPL], qsc[HG][QPL];
 #pragma unroll
         for (int h = 0; h < HG; ++h)
@@ -886,7 +897,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     }
                 }
             }
-            // Stage consumed: refill it with the item kStages ahead.
+            // Stage consumed: refill it with the item kSt ahead.
             __syncwarp();
             next_stage();
             issue_next();
