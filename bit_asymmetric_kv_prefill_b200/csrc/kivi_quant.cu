@@ -158,14 +158,27 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 constexpr int kQuantThreads = 256;
 
+// The CTA works as two independent halves: threads [0, D) take the key tile,
+// the rest the value tile, each with its own named barrier (ids 1 and 2), so
+// that neither waits for the other; the halves share only the SM.
+template <int D>
+__device__ __forceinline__ void half_sync(int tid)
+{
+    if (tid < D)
+        asm volatile("bar.sync 1, %0;" ::"n"(D) : "memory");
+    else
+        asm volatile("bar.sync 2, %0;" ::"n"(kQuantThreads - D) : "memory");
+}
+
 template <int D>
 struct QuantSmem {
     static constexpr int RS = D + 8;                      // padded row, elements
     static constexpr int TILE = 32 * RS;                  // one K or V tile
     static constexpr int TILES_BYTES = 2 * 2 * TILE * 2;  // 2 buffers x (K, V)
     static constexpr int THRK = TILES_BYTES;              // uint16 [3][D]
-    static constexpr int THRV = THRK + 3 * D * 2;         // uint16 [32][D/32][4]
-    static constexpr int OUTB = (THRV + 32 * (D / 32) * 8 + 15) / 16 * 16;
+    static constexpr int TS = 4 * (D / 32) + 4;           // padded token row of thrV
+    static constexpr int THRV = THRK + 3 * D * 2;         // uint16 [32][TS]: [D/32][4] + pad
+    static constexpr int OUTB = (THRV + 32 * TS * 2 + 15) / 16 * 16;
     static constexpr int BYTES = OUTB + 24 * D;
 };
 
@@ -182,16 +195,18 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
     const int g = (int)(item % p.n_g);
 
     if (tid < D) {
-        // Keys, per channel: thread (pair cp, row half hh) takes 16 rows of a
-        // channel pair; the halves meet through a shuffle with lane ^ 1.
+        // Keys, per channel: thread (pair cp, row set hh) takes 16 rows of a
+        // channel pair, rows 8b + 4hh + {0..3} (the two sets 4 rows apart sit
+        // in disjoint banks); they meet through a shuffle with lane ^ 1.
         const int cp = tid >> 1, hh = tid & 1;
-        const uint16_t *col = tk + hh * 16 * RS + 2 * cp;
-        uint32_t mn = *(const uint32_t *)col, mx = mn;
-        uint32_t mn1 = *(const uint32_t *)(col + RS), mx1 = mn1;
+        const uint16_t *col = tk + hh * 4 * RS + 2 * cp;
+        auto row = [&](int i) { return (const uint32_t *)(col + (((i >> 2) << 3) + (i & 3)) * RS); };
+        uint32_t mn = *row(0), mx = mn;
+        uint32_t mn1 = *row(1), mx1 = mn1;
 #pragma unroll
         for (int r = 2; r < 16; r += 2) {
-            const uint32_t v0 = *(const uint32_t *)(col + r * RS);
-            const uint32_t v1 = *(const uint32_t *)(col + (r + 1) * RS);
+            const uint32_t v0 = *row(r);
+            const uint32_t v1 = *row(r + 1);
             mn = H::vmin(mn, v0);
             mx = H::vmax(mx, v0);
             mn1 = H::vmin(mn1, v1);
@@ -228,7 +243,7 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
             mn = H::vmin(mn, (mn >> 16) | (mn << 16));
             mx = H::vmax(mx, (mx >> 16) | (mx << 16));
             const CodeParams c = code_params(H::f((uint16_t)mn), H::f((uint16_t)mx));
-            uint16_t *tr = thrV + (t * NJ + j) * 4;
+            uint16_t *tr = thrV + t * QuantSmem<D>::TS + j * 4;
             tr[0] = min_passing<DT>(c.e1, c.z);
             tr[1] = min_passing<DT>(c.e2, c.z);
             tr[2] = min_passing<DT>(c.e3, c.z);
@@ -237,7 +252,7 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
             *(uint16_t *)(outb + off + D / 16) = c.z_bits;
         }
     }
-    __syncthreads();
+    half_sync<D>(tid);
 
     if (tid < D) {
         // Key code words: thread -> (lane, token pair, word slot k); tokens tok
@@ -294,7 +309,7 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
 #pragma unroll
             for (int tt = 0; tt < TPW; ++tt) {
                 const int t = 16 * th + u * TPW + tt;
-                const uint2 tr = *(const uint2 *)(thrV + (t * NJ + j) * 4);
+                const uint2 tr = *(const uint2 *)(thrV + t * QuantSmem<D>::TS + j * 4);
                 b1[tt] = __byte_perm(tr.x, 0, 0x1010);
                 b2[tt] = __byte_perm(tr.x, 0, 0x3232);
                 b3[tt] = __byte_perm(tr.y, 0, 0x1010);
@@ -321,16 +336,24 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
             *(uint32_t *)(outb + L::VC + code_word_offset(lane, u)) = word;
         }
     }
-    __syncthreads();
+    half_sync<D>(tid);
 
+    // Each half stores its own 12*D bytes: [Kc, Km) and [Vc, Vm).
     uint4 *dst = (uint4 *)(p.packed + ((s * p.ngcap) + p.g_dst0 + g) * (long long)L::GB);
-    for (int c = tid; c < L::GB / 16; c += kQuantThreads) dst[c] = ((const uint4 *)outb)[c];
+    {
+        const int h = tid < D ? 0 : 1, ht = tid < D ? tid : tid - D;
+        const int nthr = tid < D ? D : kQuantThreads - D;
+        const uint4 *src = (const uint4 *)(outb + h * 12 * D);
+        uint4 *d = dst + h * (12 * D / 16);
+        for (int c = ht; c < 12 * D / 16; c += nthr) d[c] = src[c];
+    }
 
     if (p.newK != nullptr && g == 0) {
-        // The flush has read residual slot 0 into shared memory (the tile was
-        // complete before the first __syncthreads): the new token may land.
-        for (int c = tid; c < 2 * (D / 8); c += kQuantThreads) {
-            const int which = c / (D / 8), q = c % (D / 8);
+        // The flush has read residual slot 0 into shared memory (each half's
+        // tile was complete before that half's first barrier): the new token
+        // may land, each half writing its own row.
+        const int which = tid < D ? 0 : 1, ht = tid < D ? tid : tid - D;
+        for (int q = ht; q < D / 8; q += (tid < D ? D : kQuantThreads - D)) {
             const uint16_t *src = (which ? p.newV : p.newK) + s * D + q * 8;
             uint16_t *d = (which ? p.resV : p.resK) + s * (long long)p.R * D + q * 8;
             *(uint4 *)d = *(const uint4 *)src;
@@ -359,12 +382,14 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quant_kernel(QuantParams p)
         const long long row0 = s * p.src_seq_rows + (long long)g * 32;
         const uint16_t *k = p.srcK + row0 * D;
         const uint16_t *v = p.srcV + row0 * D;
-        uint16_t *tk = tiles + (buf * 2 + 0) * S::TILE;
-        uint16_t *tv = tiles + (buf * 2 + 1) * S::TILE;
-        for (int c = tid; c < 32 * (D / 8); c += kQuantThreads) {
+        // The key half copies the key tile, the value half the value tile.
+        const bool kh = tid < D;
+        uint16_t *t = tiles + (buf * 2 + (kh ? 0 : 1)) * S::TILE;
+        const uint16_t *src = kh ? k : v;
+        const int ht = kh ? tid : tid - D, nthr = kh ? D : kQuantThreads - D;
+        for (int c = ht; c < 32 * (D / 8); c += nthr) {
             const int row = c / (D / 8), col = (c % (D / 8)) * 8;
-            cp_async16(tk + row * S::RS + col, k + row * D + col);
-            cp_async16(tv + row * S::RS + col, v + row * D + col);
+            cp_async16(t + row * S::RS + col, src + row * D + col);
         }
     };
 
@@ -376,7 +401,7 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quant_kernel(QuantParams p)
         issue(item + gridDim.x, buf ^ 1);
         cp_async_commit();
         cp_async_wait<1>();
-        __syncthreads();
+        half_sync<D>(tid);
         if (item < n_group_items) {
             quantize_tile<D, DT>(p, item, tiles + (buf * 2 + 0) * S::TILE,
                                  tiles + (buf * 2 + 1) * S::TILE, thrK, thrV, outb);
@@ -388,12 +413,12 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quant_kernel(QuantParams p)
             const uint4 *sv = (const uint4 *)(p.srcV + (s * p.src_seq_rows + p.copy_row0) * D);
             uint4 *dk = (uint4 *)(p.resK + s * (long long)p.R * D);
             uint4 *dv = (uint4 *)(p.resV + s * (long long)p.R * D);
-            for (long long c = tid; c < n16; c += kQuantThreads) {
-                dk[c] = sk[c];
-                dv[c] = sv[c];
-            }
+            const bool kh = tid < D;
+            const uint4 *sr = kh ? sk : sv;
+            uint4 *dr = kh ? dk : dv;
+            for (long long c = kh ? tid : tid - D; c < n16; c += kh ? D : kQuantThreads - D) dr[c] = sr[c];
         }
-        __syncthreads();
+        half_sync<D>(tid);
     }
     cp_async_wait<0>();
 }
