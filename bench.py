@@ -15,6 +15,11 @@ bytes / CUDA-event duration of each launch) is reported against the measured
 copy bandwidth in MEASURED_PEAKS.json.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME] [--batch B] [--decode-steps S] [--layers L]
+
+The default workload is the Llama-2-7B layer above; `--workload` times any
+other workload of synth.WORKLOADS the same way (a step being its prefill and
+decode steps), `--batch` and `--decode-steps` shrink it.
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own replica
 (no data exchange: sequences and heads are independent) and the reported value
@@ -64,6 +69,21 @@ def decode_schedule(w):
     return out
 
 
+def get_workload(args):
+    from bit_asymmetric_kv_prefill_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    over = {}
+    if args.batch:
+        over["B"] = args.batch
+    if args.decode_steps:
+        over["steps"] = args.decode_steps
+    return synth.scaled(w, **over) if over else w
+
+
+def is_headline(args):
+    return args.workload == WORKLOAD and not args.batch and not args.decode_steps
+
+
 def decode_bytes(w, n_q, r):
     """Algorithmic HBM bytes of one decode call: per quantized (token, kv head)
     the 2-bit K and V codes plus fp16 scale/zero (D/4 + 4D/G for each of K and
@@ -94,9 +114,11 @@ def measured_peak():
         return 6650.0, "fallback"
 
 
-def traffic_per_launch():
+def traffic_per_launch(args):
     """dram read+write bytes per decode launch from the committed ncu summary,
-    or None when absent or taken on other kernel sources."""
+    or None when absent, taken on other kernel sources or on another workload."""
+    if not is_headline(args):
+        return None
     try:
         with open(PROFILE_TRAFFIC) as f:
             d = json.load(f)
@@ -216,7 +238,8 @@ def oracle_stream_rate(w, seconds: float, max_seqs: int = 1 << 30):
         kb, vb = synth.bits(K), synth.bits(V)
         steps = [tuple(synth.bits(x) for x in synth.step_inputs(one, s, seed=done))
                  for s in range(1, w.steps + 1)]
-        c = oracle.OracleCache(1, 1, w.D, w.G, w.R, dt, w.T_max)
+        c = oracle.OracleCache(1, 1, w.D, w.G, w.R, dt, w.T_max, pre_rope=w.pre_rope,
+                               rope_theta=w.rope_theta)
         t0 = time.perf_counter()
         c.prefill(kb, vb)
         for k, v, q in steps:
@@ -234,7 +257,7 @@ def run_reference(args):
     import oracle
     from bit_asymmetric_kv_prefill_b200 import synth
     oracle.build()
-    w = synth.WORKLOADS[WORKLOAD]
+    w = get_workload(args)
     for _ in range(args.warmup):
         oracle_stream_rate(w, 0.0, max_seqs=1)
     t_total, units_total = 0.0, 0.0
@@ -244,7 +267,7 @@ def run_reference(args):
         t_total += t
         units_total += units_seq * n
     value = units_total / t_total
-    sample = (f"each step: one (batch, head) sequence of {WORKLOAD}: prefill T={w.T} + "
+    sample = (f"each step: one (batch, head) sequence of {w.name}: prefill T={w.T} + "
               f"{w.steps} x (append + decode), single thread")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
@@ -260,13 +283,19 @@ def run_reference(args):
 # ---- GPU leg ----------------------------------------------------------------------------
 
 def workload_config(w, args):
-    return {"workload": f"{WORKLOAD}: Llama-2-7B layer shape, batch {w.B}, {w.H_q} MHA heads, "
-                        f"head_dim {w.D}, context {w.T}, G={w.G}, R={w.R}, bf16 input/residual, "
+    heads = f"{w.H_q} MHA heads" if w.H_q == w.H_kv else f"{w.H_q} query heads over {w.H_kv} kv heads"
+    title = "Llama-2-7B layer shape, " if w.name == WORKLOAD else ""
+    rope = f", keys pre-RoPE (theta {w.rope_theta:g})" if w.pre_rope else ""
+    per_layer = w.B * w.H_kv * (w.T_max * 2 * (w.D // 4 + 4 * w.D // w.G) + w.R * 4 * w.D)
+    ws_mb = args.layers * per_layer / 1e6
+    l2 = (f"inputs larger than L2: {args.layers} layer caches visited round-robin "
+          f"(~{ws_mb:.0f} MB working set vs 126 MB L2), no explicit flush") if ws_mb > 126 else \
+         f"working set {ws_mb:.0f} MB, not larger than L2 (126 MB)"
+    return {"workload": f"{w.name}: {title}batch {w.B}, {heads}, head_dim {w.D}, context {w.T}, "
+                        f"G={w.G}, R={w.R}, {w.dtype} input/residual{rope}, "
                         f"prefill + {w.steps} x (append + decode) per layer",
             "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "D": w.D, "T": w.T, "G": w.G, "R": w.R,
-            "decode_steps": w.steps, "layers_round_robin": args.layers,
-            "l2": f"inputs larger than L2: {args.layers} layer caches visited round-robin "
-                  f"(~{args.layers * 134} MB working set vs 126 MB L2), no explicit flush",
+            "decode_steps": w.steps, "layers_round_robin": args.layers, "l2": l2,
             "parallelism": f"replicas x{max(1, args.gpus)} (no data-path collective)"}
 
 
@@ -287,14 +316,15 @@ def run_gpu(args):
     kbuild.build()
     L = kivi.lib()
 
-    w = synth.WORKLOADS[WORKLOAD]
+    w = get_workload(args)
     nl = args.layers
     sched = decode_schedule(w)
     bytes_step = sum(decode_bytes(w, n, r) for n, r in sched) * nl
     units_step = sum(decode_units(w, n, r) for n, r in sched) * nl
     launches_step = nl * (1 + 2 * w.steps)
 
-    caches = [KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, w.T_max) for _ in range(nl)]
+    caches = [KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, w.T_max, pre_rope=w.pre_rope,
+                        rope_theta=w.rope_theta) for _ in range(nl)]
     Ks, Vs = [], []
     for l in range(nl):
         K, V = synth.prefill_inputs(w, seed=1000 * rank + l, device=dev)
@@ -364,7 +394,7 @@ def run_gpu(args):
     bytes_per_launch = bytes_step / n_dec
     achieved = bytes_per_launch / (dec_avg / 1e3) / 1e9
     peak, peak_kind = measured_peak()
-    traffic = traffic_per_launch()
+    traffic = traffic_per_launch(args)
 
     e2e = run_e2e(args, w, caches, Ks, Vs, steps, dev, world)
 
@@ -372,7 +402,7 @@ def run_gpu(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, nseq, secs = oracle_stream_rate(w, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{nseq} (batch, head) sequences of {WORKLOAD}, each prefill T={w.T} + "
+               "sample": f"{nseq} (batch, head) sequences of {w.name}, each prefill T={w.T} + "
                          f"{w.steps} x (append + decode); {secs:.1f} s single-threaded"}
 
     if rank == 0:
@@ -459,6 +489,11 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", dest="e2e_steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", dest="cpu_seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", dest="no_cpu_baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=["tiny", "llama2_7b_layer", "llama2_13b_cache", "mistral_gqa", "long_context"])
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
+    ap.add_argument("--decode-steps", dest="decode_steps", type=int, default=0,
+                    help="override the workload's decode steps")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
