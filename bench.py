@@ -3,7 +3,8 @@
 One step = one pass of the whole hot path over the Llama-2-7B layer workload
 (batch 8, 32 MHA heads, head_dim 128, 4,096-token context, G=32, R=128, bf16):
 prefill quantization, then 64 decode steps each appending one token (the first
-append flushes the full residual) and running decode attention.  The step runs
+append flushes the full residual) and running decode attention, the append fused
+into the decode launch (kivi_append_decode) except where it flushes.  The step runs
 over `--layers` independent layer caches (default 8) visited round-robin, as a
 model's decode does, so the working set (~1.1 GB) is far larger than the
 126 MB L2 and every decode streams its cache from HBM.
@@ -82,6 +83,13 @@ def get_workload(args):
 
 def is_headline(args):
     return args.workload == WORKLOAD and not args.batch and not args.decode_steps
+
+
+def flush_steps(w):
+    """Per decode step, whether its append flushes the residual (n_q grows)."""
+    sched = decode_schedule(w)
+    n_q0 = w.R * ((w.T - 1) // w.R)
+    return [sched[j][0] != (sched[j - 1][0] if j else n_q0) for j in range(w.steps)]
 
 
 def decode_bytes(w, n_q, r):
@@ -319,9 +327,11 @@ def run_gpu(args):
     w = get_workload(args)
     nl = args.layers
     sched = decode_schedule(w)
-    bytes_step = sum(decode_bytes(w, n, r) for n, r in sched) * nl
+    # A fused launch also reads k_t, v_t and writes them to the residual.
+    fused_extra = 4 * w.B * w.H_kv * w.D * 2 * (w.steps - sum(flush_steps(w)))
+    bytes_step = (sum(decode_bytes(w, n, r) for n, r in sched) + fused_extra) * nl
     units_step = sum(decode_units(w, n, r) for n, r in sched) * nl
-    launches_step = nl * (1 + 2 * w.steps)
+    launches_step = nl * (1 + w.steps + sum(flush_steps(w)))
 
     caches = [KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, w.T_max, pre_rope=w.pre_rope,
                         rope_theta=w.rope_theta) for _ in range(nl)]
@@ -341,8 +351,12 @@ def run_gpu(args):
     Sp = [[tuple(ctypes.c_void_p(t.data_ptr()) for t in st) for st in row] for row in steps]
     Op = [ctypes.c_void_p(o.data_ptr()) for o in outs]
     T, Hq = w.T, w.H_q
-    reset, prefill, append, decode = (L.kivi_cache_reset, L.kivi_prefill, L.kivi_append,
-                                      L.kivi_decode_attn)
+    reset, prefill, append, decode, fused = (L.kivi_cache_reset, L.kivi_prefill, L.kivi_append,
+                                             L.kivi_decode_attn, L.kivi_append_decode)
+    # Steps whose append flushes (the quantizer runs): append, then decode;
+    # the others fuse the append into the decode launch.  Either way the timed
+    # launch is one decode.
+    flush = flush_steps(w)
 
     def one_step(ev=None):
         bad = 0
@@ -350,13 +364,17 @@ def run_gpu(args):
             bad |= reset(H[l])
             bad |= prefill(H[l], Kp[l], Vp[l], T, sp)
         i = 0
-        for row in Sp:
+        for j, row in enumerate(Sp):
             for l in range(nl):
                 k, v, q = row[l]
-                bad |= append(H[l], k, v, sp)
+                if flush[j]:
+                    bad |= append(H[l], k, v, sp)
                 if ev is not None:
                     ev[i][0].record(stream)
-                bad |= decode(H[l], q, Hq, Op[l], sp)
+                if flush[j]:
+                    bad |= decode(H[l], q, Hq, Op[l], sp)
+                else:
+                    bad |= fused(H[l], k, v, q, Hq, Op[l], sp)
                 if ev is not None:
                     ev[i][1].record(stream)
                 i += 1
@@ -455,8 +473,7 @@ def run_e2e(args, w, caches, Ks, Vs, steps, dev, world):
         for row in hS:
             for l in range(nl):
                 k, v, q = (d.copy_(h, non_blocking=True) for d, h in zip(dS[l], row[l]))
-                caches[l].append(k, v)
-                out = caches[l].decode(q)
+                out = caches[l].append_decode(k, v, q)
                 hout[l].copy_(out, non_blocking=True)
 
     n = max(1, min(args.steps, args.e2e_steps))

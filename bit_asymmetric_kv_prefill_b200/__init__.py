@@ -72,6 +72,7 @@ def lib():
     L.kivi_prefill.argtypes = [vp, vp, vp, i64, vp]
     L.kivi_append.argtypes = [vp, vp, vp, vp]
     L.kivi_decode_attn.argtypes = [vp, vp, i32, vp, vp]
+    L.kivi_append_decode.argtypes = [vp, vp, vp, vp, i32, vp, vp]
     L.kivi_decode_attn_noalloc.argtypes = [vp, vp, i32, vp, vp]
     L.kivi_cache_reset.argtypes = [vp]
     L.kivi_cache_length.argtypes = [vp, P(i64), P(i32)]
@@ -82,6 +83,7 @@ def lib():
     L.kivi_decode_split.argtypes = [i64, i64, i32, i32, i32, i64, i64, i64, P(i64)]
     for name in ("kivi_cache_create", "kivi_cache_create_ex", "kivi_cache_required_bytes",
                  "kivi_prefill", "kivi_append", "kivi_decode_attn", "kivi_decode_attn_noalloc",
+                 "kivi_append_decode",
                  "kivi_cache_reset",
                  "kivi_cache_length", "kivi_cache_bytes", "kivi_export", "kivi_device_status",
                  "kivi_cache_destroy", "kivi_decode_split"):
@@ -197,6 +199,22 @@ class KiviCache:
             raise ValueError("out must be a contiguous CUDA float32 [B, H_q, D] tensor")
         _check(lib().kivi_decode_attn(self._h, qp, H_q, out.data_ptr(), _stream_ptr(stream)),
                "kivi_decode_attn")
+        return out
+
+    def append_decode(self, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor,
+                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+        """append(k, v) then decode(q) in one launch (two when a flush is due)."""
+        shape = (self.B, self.H_kv, self.D)
+        kp, vp_ = self._tensor(k, shape, "k_t"), self._tensor(v, shape, "v_t")
+        H_q = q.shape[1]
+        qp = self._tensor(q, (self.B, H_q, self.D), "q")
+        if out is None:
+            out = torch.empty((self.B, H_q, self.D), dtype=torch.float32, device=q.device)
+        elif (out.dtype != torch.float32 or tuple(out.shape) != (self.B, H_q, self.D)
+              or not out.is_contiguous() or not out.is_cuda):
+            raise ValueError("out must be a contiguous CUDA float32 [B, H_q, D] tensor")
+        _check(lib().kivi_append_decode(self._h, kp, vp_, qp, H_q, out.data_ptr(), _stream_ptr(stream)),
+               "kivi_append_decode")
         return out
 
     def decode_noalloc(self, q: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:

@@ -327,6 +327,38 @@ kivi_status kivi_append(kivi_cache *c, const void *k_t, const void *v_t, void *s
     return KIVI_OK;
 }
 
+kivi_status kivi_append_decode(kivi_cache *c, const void *k_t, const void *v_t, const void *q,
+                               int H_q, float *out, void *stream)
+{
+    if (!c || !k_t || !v_t || !aligned16(k_t) || !aligned16(v_t)) return KIVI_ERR_ARG;
+    if (!c->prefilled) return KIVI_ERR_STATE;
+    if (c->n_q + c->r + 1 > c->cfg.T_max) return KIVI_ERR_CAPACITY;
+    if (c->r == c->cfg.R) {   // a flush is due: the quantizer runs first
+        const kivi_status st = kivi_append(c, k_t, v_t, stream);
+        return st != KIVI_OK ? st : kivi_decode_attn(c, q, H_q, out, stream);
+    }
+    // The split sees the token already appended; undone if anything fails
+    // before the launch.
+    c->r += 1;
+    DecodeParams p;
+    int D = 0, HG = 0, dtype = 0, pre_rope = 0;
+    kivi_status st = decode_params_external_scratch(c, q, H_q, out, &p, &D, &HG, &dtype, &pre_rope);
+    if (st == KIVI_OK && p.slots > c->plan.slots) st = KIVI_ERR_UNSUPPORTED;
+    if (st != KIVI_OK) {
+        c->r -= 1;
+        return st;
+    }
+    p.partials = c->partials;
+    p.tickets = c->tickets;
+    p.slots = c->plan.slots;
+    p.newK = (const uint16_t *)k_t;
+    p.newV = (const uint16_t *)v_t;
+    p.new_slot = c->r - 1;
+    const cudaError_t e = launch_decode(D, HG, dtype, pre_rope, p, (cudaStream_t)stream);
+    if (e != cudaSuccess) c->r -= 1;
+    return cuda_status(e);
+}
+
 kivi_status kivi_decode_attn(kivi_cache *c, const void *q, int H_q, float *out, void *stream)
 {
     DecodeParams p;
@@ -526,6 +558,8 @@ kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q
     p->slots = (int)(warps / p->seqs + 2);
     p->qscale = (float)(1.4426950408889634 / std::sqrt((double)c->cfg.D));
     p->inv_freq = c->inv_freq;
+    p->newK = p->newV = nullptr;
+    p->new_slot = -1;
     p->magic = 0x4B000000u;
     p->neg_magic = -8388608.0f;
     *D = c->cfg.D;

@@ -420,8 +420,27 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
             const int nt = min(kResTok, p.r - t0);
             const uint32_t bytes = (uint32_t)nt * D * 2;
             const long long row = (long long)pf_s * p.R + t0;
-            lane0_expect_copy(lane, bar, dst, p.resK + row * D, bytes, 2 * bytes);
-            lane0_copy(lane, bar, dst + kResTok * D * 2, p.resV + row * D, bytes);
+            const int nn = p.new_slot - t0;   // the appended token's row in this slice
+            if (p.newK != nullptr && nn >= 0 && nn < nt) {
+                // Fused append: the slice's last row comes from the caller's
+                // k_t/v_t (slot new_slot, the residual's newest); the rows
+                // before it from the residual.
+                const uint32_t head = (uint32_t)nn * D * 2;
+                lane0_expect_copy(lane, bar, dst + head, p.newK + (long long)pf_s * D, D * 2, 2 * bytes);
+                lane0_copy(lane, bar, dst + kResTok * D * 2 + head, p.newV + (long long)pf_s * D, D * 2);
+                if (nn > 0) {
+                    lane0_copy(lane, bar, dst, p.resK + row * D, head);
+                    lane0_copy(lane, bar, dst + kResTok * D * 2, p.resV + row * D, head);
+                }
+                if (nn + 1 < nt) {   // (the appended token is the newest: never taken)
+                    const uint32_t tail = (uint32_t)(nt - nn - 1) * D * 2;
+                    lane0_copy(lane, bar, dst + head + D * 2, p.resK + (row + nn + 1) * D, tail);
+                    lane0_copy(lane, bar, dst + kResTok * D * 2 + head + D * 2, p.resV + (row + nn + 1) * D, tail);
+                }
+            } else {
+                lane0_expect_copy(lane, bar, dst, p.resK + row * D, bytes, 2 * bytes);
+                lane0_copy(lane, bar, dst + kResTok * D * 2, p.resV + row * D, bytes);
+            }
         }
         ++issued;
         ++pf_i;
@@ -822,6 +841,18 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 const int nt = min(kResTok, p.r - t0);
                 const uint16_t *rk = (const uint16_t *)st;
                 const uint16_t *rv = (const uint16_t *)(st + kResTok * D * 2);
+                if (p.newK != nullptr && p.new_slot >= t0 && p.new_slot < t0 + nt) {
+                    // Fused append: this warp persists the new token into its
+                    // residual slot (read by later launches' bulk copies).
+                    constexpr int C16 = D / 8;   // 16-byte chunks per row
+                    const int nn = p.new_slot - t0;
+                    const long long drow = ((long long)s * p.R + p.new_slot) * D;
+                    for (int c = lane; c < 2 * C16; c += 32) {
+                        const int which = c / C16, q16 = c % C16;
+                        const uint4 v = *(const uint4 *)((which ? rv : rk) + nn * D + q16 * 8);
+                        *(uint4 *)((which ? p.resV : p.resK) + drow + q16 * 8) = v;
+                    }
+                }
                 const bool valid = tq < nt;
                 float sc[HG];
                 {

@@ -51,6 +51,10 @@ struct DecodeParams {
     uint32_t magic;      // bits of 2^23 (the code-to-float exponent)
     float neg_magic;     // -2^23
     const float *inv_freq;  // RoPE inverse frequencies [D/2] (pre-RoPE caches)
+    // Fused append: the token at residual slot new_slot is read from newK /
+    // newV ([seqs][D]) and stored to the residual by the decode (else null, -1).
+    const uint16_t *newK, *newV;
+    int new_slot;
 };
 
 int num_sms();

@@ -136,6 +136,15 @@ KIVI_API kivi_status kivi_append(kivi_cache *c, const void *k_t, const void *v_t
 KIVI_API kivi_status kivi_decode_attn(kivi_cache *c, const void *q, int H_q, float *out,
                              void *stream);
 
+/* kivi_append then kivi_decode_attn in one launch (the pages have no
+ * counterpart; this is the decode step of a model, fused): the decode reads
+ * the appended token from k_t/v_t and stores it to the residual itself.  When
+ * the residual is full (a flush is due) it runs the two calls.  Arguments,
+ * layouts and errors are those of the two calls; on an error before the
+ * launch the cache is unchanged. */
+KIVI_API kivi_status kivi_append_decode(kivi_cache *c, const void *k_t, const void *v_t,
+                               const void *q, int H_q, float *out, void *stream);
+
 /*
  * Decode attention exactly as kivi_decode_attn, for callers that must not
  * allocate device memory (no part of the method corresponds to this call: it

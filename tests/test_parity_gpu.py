@@ -186,6 +186,60 @@ def test_lossless_cache_matches_textbook_attention():
         assert np.all(err <= bound + 1e-6 * np.abs(ref).max()), float((err - bound).max())
 
 
+# ---- fused append + decode -----------------------------------------------------------
+
+FUSED = [
+    ("tiny", dict(T=130, B=2, H_q=4, H_kv=2), 140),          # crosses a flush
+    ("tiny", dict(T=31, B=1, dtype="bf16"), 40),              # D = 64
+    ("llama2_7b_layer", dict(B=2, H_q=2, H_kv=2, T=300), 30),
+    ("mistral_gqa", dict(B=2, H_q=8, H_kv=2, T=257, R=64), 70),
+    ("long_context", dict(B=1, H_q=8, H_kv=2, T=200), 60),   # pre-RoPE
+]
+
+
+@pytest.mark.parametrize("name,kw,steps", FUSED,
+                         ids=[f"{n}-{'-'.join(f'{k}{v}' for k, v in kw.items())}" for n, kw, _ in FUSED])
+def test_append_decode_equals_append_then_decode(name, kw, steps):
+    """The fused call gives the separate calls' outputs bit for bit and leaves
+    the same cache behind, flushes included."""
+    w = small(name, steps=steps, **kw)
+    K, V = synth.prefill_inputs(w, 9, device=DEV)
+    mk = lambda: KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, w.T_max,
+                           pre_rope=w.pre_rope, rope_theta=w.rope_theta)
+    a, b = mk(), mk()
+    a.prefill(K, V)
+    b.prefill(K, V)
+    for s in range(1, steps + 1):
+        k, v, q = synth.step_inputs(w, s, 9, device=DEV)
+        a.append(k, v)
+        oa = a.decode(q)
+        ob = b.append_decode(k, v, q)
+        assert a.length() == b.length()
+        assert torch.equal(oa, ob), f"step {s}"
+    ea, eb = a.export(), b.export()
+    for key in ea:
+        assert np.array_equal(ea[key], eb[key]), key
+    assert a.device_status() == 0 and b.device_status() == 0
+
+
+def test_append_decode_rejects_bad_arguments():
+    w = small("tiny", T=40, steps=0)
+    K, V = synth.prefill_inputs(w, 0, device=DEV)
+    c = KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, T_max=41)
+    k, v, q = synth.step_inputs(w, 1, 0, device=DEV)
+    with pytest.raises(KiviError):
+        c.append_decode(k, v, q)                 # before prefill
+    c.prefill(K, V)
+    with pytest.raises(KiviError):               # 3 query heads over 2 kv heads
+        c.append_decode(k, v, torch.zeros(w.B, 3, w.D, dtype=q.dtype, device=DEV))
+    assert c.length() == (0, 40)                 # unchanged by the failed call
+    c.append_decode(k, v, q)
+    assert c.length() == (0, 41)
+    with pytest.raises(KiviError):
+        c.append_decode(k, v, q)                 # past T_max
+    assert c.device_status() == 0
+
+
 # ---- argument and state errors -----------------------------------------------------
 
 def test_errors_and_capacity():
