@@ -48,11 +48,15 @@ namespace kivi {
 #ifndef KIVI_DECODE_MAXW_GQA
 #define KIVI_DECODE_MAXW_GQA 12   // four or more query heads per kv head
 #endif
+#ifndef KIVI_ROPE_UNROLL
+#define KIVI_ROPE_UNROLL 1   // pre-RoPE key loop: pair-steps unrolled (measured best)
+#endif
 #ifndef KIVI_SCALAR_F32
 #define KIVI_SCALAR_F32 0
 #endif
 
 constexpr unsigned FULL = 0xffffffffu;
+constexpr int kRopeUnroll = KIVI_ROPE_UNROLL;
 #ifndef KIVI_DECODE_STAGES_GQA
 #define KIVI_DECODE_STAGES_GQA 3   // four or more query heads per kv head
 #endif
@@ -651,33 +655,34 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                         for (int h = 0; h < HG; ++h) part[t][h] = acc[t][h].x + acc[t][h].y;
                 } else {
                     // Dequantize, rotate at absolute positions, dot with q, two
-                    // rotate-half pairs (i, i+1) of the slice at a time.
+                    // rotate-half pairs (i, i+1) of the slice at a time, each
+                    // pair's scale/zero, frequencies and query pairs loaded once
+                    // for the lane's 4 tokens.
                     const long long tbase = (long long)it * kG + 4 * tq;
-#pragma unroll 1
-                    for (int t = 0; t < 4; ++t) {
-                        const float pos = (float)(tbase + t);
-                        // Token t's words, picked by selects (an index by the
-                        // rolled t would move kw to the stack).
-                        uint32_t wt[KW];
+                    float d0[4][HG], d1[4][HG];
 #pragma unroll
-                        for (int k = 0; k < KW; ++k)
-                            wt[k] = t == 0 ? kw[k] : t == 1 ? kw[KW + k] : t == 2 ? kw[2 * KW + k] : kw[3 * KW + k];
-                        float d0[HG], d1[HG];
+                    for (int t = 0; t < 4; ++t)
 #pragma unroll
-                        for (int h = 0; h < HG; ++h) d0[h] = d1[h] = 0.f;
-#pragma unroll 2
-                        for (int i = 0; i < HALF; i += 2) {
-                            // Local channels i, i+1 (first RoPE half) and HALF+i,
-                            // HALF+i+1 (their partners); word k = L/16, pair (L%16)/2.
-                            const int Lx = i, Ly = HALF + i;
-                            const uint32_t wx = wt[Lx / 16], wy = wt[Ly / 16];
+                        for (int h = 0; h < HG; ++h) d0[t][h] = d1[t][h] = 0.f;
+#pragma unroll kRopeUnroll
+                    for (int i = 0; i < HALF; i += 2) {
+                        // Local channels i, i+1 (first RoPE half) and HALF+i,
+                        // HALF+i+1 (their partners); word k = L/16, pair (L%16)/2.
+                        const int Lx = i, Ly = HALF + i;
+                        const float4 sx = *(const float4 *)(sz + cs * W::SZS + Lx);
+                        const float4 sy = *(const float4 *)(sz + cs * W::SZS + Ly);
+                        const float2 f2 = *(const float2 *)(frq + cs * W::FRS + i);
+                        float4 qq[HG];
+#pragma unroll
+                        for (int h = 0; h < HG; ++h) qq[h] = *(const float4 *)(qr + (h * 4 + cs) * W::QRS + i);
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const float pos = (float)(tbase + t);
+                            const uint32_t wx = kw[t * KW + Lx / 16], wy = kw[t * KW + Ly / 16];
                             const float2 cx = code_pair(wx, wx >> 16, (Lx % 16) / 2, magic, neg);
                             const float2 cy = code_pair(wy, wy >> 16, (Ly % 16) / 2, magic, neg);
-                            const float4 sx = *(const float4 *)(sz + cs * W::SZS + Lx);
-                            const float4 sy = *(const float4 *)(sz + cs * W::SZS + Ly);
                             const float x0 = fmaf(cx.x, sx.x, sx.y), x1 = fmaf(cx.y, sx.z, sx.w);
                             const float y0 = fmaf(cy.x, sy.x, sy.y), y1 = fmaf(cy.y, sy.z, sy.w);
-                            const float2 f2 = *(const float2 *)(frq + cs * W::FRS + i);
                             float sn0, cn0, sn1, cn1;
                             rope_sincos(__fmul_rn(pos, f2.x), &sn0, &cn0);
                             rope_sincos(__fmul_rn(pos, f2.y), &sn1, &cn1);
@@ -685,21 +690,17 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                             const float rx1 = x1 * cn1 - y1 * sn1, ry1 = y1 * cn1 + x1 * sn1;
 #pragma unroll
                             for (int h = 0; h < HG; ++h) {
-                                const float4 qq = *(const float4 *)(qr + (h * 4 + cs) * W::QRS + i);
-                                d0[h] = fmaf(qq.x, rx0, d0[h]);
-                                d1[h] = fmaf(qq.y, ry0, d1[h]);
-                                d0[h] = fmaf(qq.z, rx1, d0[h]);
-                                d1[h] = fmaf(qq.w, ry1, d1[h]);
+                                d0[t][h] = fmaf(qq[h].x, rx0, d0[t][h]);
+                                d1[t][h] = fmaf(qq[h].y, ry0, d1[t][h]);
+                                d0[t][h] = fmaf(qq[h].z, rx1, d0[t][h]);
+                                d1[t][h] = fmaf(qq[h].w, ry1, d1[t][h]);
                             }
                         }
-#pragma unroll
-                        for (int h = 0; h < HG; ++h) {
-                            const float d = d0[h] + d1[h];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                if (u == t) part[u][h] = d;
-                        }
                     }
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+#pragma unroll
+                        for (int h = 0; h < HG; ++h) part[t][h] = d0[t][h] + d1[t][h];
                 }
                 // Transpose-reduce the 4 token partials over the 4 slices: lane
                 // (tq, cs) ends with token 4tq + cs = lane.
