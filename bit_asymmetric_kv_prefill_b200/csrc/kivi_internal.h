@@ -26,6 +26,7 @@ struct QuantParams {
     int r_copy;                   // prefill: residual rows to copy (0: none)
     long long copy_row0;          // prefill: first source row of the residual
     const uint16_t *newK, *newV;  // flush: token to store in slot 0 (or null)
+    Magic div_ng;                 // division by n_g (set by launch_quant)
 };
 
 struct DecodeParams {

@@ -83,9 +83,11 @@ struct In<0> {  // IEEE fp16
 template <int DT>
 __device__ __forceinline__ uint16_t next_up(uint16_t b)
 {
-    if ((b & 0x7fffu) == 0) return 0x0001u;
-    if (b & 0x8000u) return (uint16_t)(b - 1);
-    return b == In<DT>::kInf ? b : (uint16_t)(b + 1);
+    // Value order: +-0 -> smallest positive subnormal, negatives step towards
+    // zero, positives away from it, +inf stays (selects, no branches).
+    const uint16_t up = (b & 0x8000u) ? (uint16_t)(b - 1) : (uint16_t)(b + 1);
+    const uint16_t r = (b & 0x7fffu) == 0 ? (uint16_t)0x0001u : up;
+    return b == In<DT>::kInf ? b : r;
 }
 template <int DT>
 __device__ __forceinline__ uint16_t next_down(uint16_t b)
@@ -110,12 +112,26 @@ __device__ __forceinline__ bool passes(uint16_t x, float e, float z)
 // steps.  Should that not happen within 4 steps, a binary search over the
 // value-ordered 16-bit patterns settles it.
 template <int DT>
+__device__ __noinline__ uint16_t min_passing_slow(uint16_t x, float e, float z);
+
+template <int DT>
 __device__ __forceinline__ uint16_t min_passing(float e, float z)
 {
     if (!(e < __int_as_float(0x7f800000))) return In<DT>::kInf;
-    uint16_t x = In<DT>::from_float_rd(__fadd_rd(z, e));
+    // The first two steps, evaluated side by side; rarely more are needed.
+    const uint16_t x0 = In<DT>::from_float_rd(__fadd_rd(z, e));
+    const uint16_t x1 = next_up<DT>(x0), x2 = next_up<DT>(x1);
+    const bool p1 = passes<DT>(x1, e, z), p2 = passes<DT>(x2, e, z);
+    if (p1 | p2) return p1 ? x1 : x2;
+    return min_passing_slow<DT>(x2, e, z);
+}
+
+// Continuation from x (not passing): two more steps, then a bisection.
+template <int DT>
+__device__ __noinline__ uint16_t min_passing_slow(uint16_t x, float e, float z)
+{
 #pragma unroll 1
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
         x = next_up<DT>(x);
         if (passes<DT>(x, e, z)) return x;
     }
@@ -191,8 +207,8 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
     constexpr int RS = QuantSmem<D>::RS;
     constexpr int NJ = L::NJ, CPL = L::CPL, TPW = L::TPW, KW = L::KW;
     const int tid = threadIdx.x;
-    const long long s = item / p.n_g;
-    const int g = (int)(item % p.n_g);
+    const long long s = div_floor(item, p.div_ng);
+    const int g = (int)(item - s * p.n_g);
 
     if (tid < D) {
         // Keys, per channel: thread (pair cp, row set hh) takes 16 rows of a
@@ -377,8 +393,8 @@ __global__ void __launch_bounds__(kQuantThreads, 3) quant_kernel(QuantParams p)
 
     auto issue = [&](long long item, int buf) {
         if (item >= n_group_items) return;
-        const long long s = item / p.n_g;
-        const int g = (int)(item % p.n_g);
+        const long long s = div_floor(item, p.div_ng);
+        const int g = (int)(item - s * p.n_g);
         const long long row0 = s * p.src_seq_rows + (long long)g * 32;
         const uint16_t *k = p.srcK + row0 * D;
         const uint16_t *v = p.srcV + row0 * D;
@@ -463,7 +479,9 @@ static cudaError_t launch_quant_t(const QuantParams &p, cudaStream_t st)
     if (items == 0) return cudaSuccess;
     long long grid = (long long)num_sms() * 3;
     if (grid > items) grid = items;
-    quant_kernel<D, DT><<<(unsigned)grid, kQuantThreads, S::BYTES, st>>>(p);
+    QuantParams q = p;
+    q.div_ng = make_magic((unsigned long long)(p.n_g > 0 ? p.n_g : 1));
+    quant_kernel<D, DT><<<(unsigned)grid, kQuantThreads, S::BYTES, st>>>(q);
     return cudaGetLastError();
 }
 
