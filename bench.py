@@ -106,10 +106,18 @@ def decode_units(w, n_q, r):
 
 
 def source_hash():
+    """sha256 of the decode kernel's sources with comments and blank lines
+    removed (an edit of comments leaves the compiled kernel, and so the
+    recorded counters, as they were)."""
+    import re
     h = hashlib.sha256()
     for rel in DECODE_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
+        h.update("\n".join(lines).encode())
     return h.hexdigest()
 
 

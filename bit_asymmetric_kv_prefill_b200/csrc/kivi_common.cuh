@@ -37,8 +37,10 @@ constexpr long long kRopeMaxTokens = 823000;
 // at bits [2i, 2i+1] and its second at bits [16+2i, 17+2i].  In a K word pair
 // i is local channels (16k+2i, 16k+2i+1); in a V word pair i is token
 // 16th + u*TPW + i/(CPL/2), channels co*CPL + 2*(i%(CPL/2)) and the next one.
-// Both halves of a pair sit at the same shift, so a decoder reads the pair from
-// the word and from the word shifted right by 16 with one logic op per code.
+// Both halves of a pair sit at the same shift, so one mask reads both: from
+// the word and from the word shifted right by 16 (keys, one logic op per
+// code), or as the two 16-bit halves of one register (values, one logic op
+// per pair).
 // ---------------------------------------------------------------------------
 template <int D>
 struct Layout {

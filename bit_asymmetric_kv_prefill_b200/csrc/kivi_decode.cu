@@ -15,12 +15,14 @@
 //    mbarriers; every wait is bounded and reports through the status word.
 //  * Keys: per group the lane folds the per-channel scale into the query,
 //    q'_d = q_d * s_d, and the zero into one bias b = sum_d q_d z_d, so that
-//    q.k = sum_d q'_d c_d + b.  Codes are turned into floats by OR-ing the
-//    2-bit field into a float's mantissa under a fixed exponent and
-//    subtracting the exponent's power of two (exact), two at a time with
-//    packed fp32x2 adds and FMAs.
-//  * Values: p'_{t,j} = p_t s_{t,j} and sum_t p_t z_{t,j} likewise fold the
-//    per-token scale and zero; lanes own channels.
+//    q.k = sum_d q'_d c_d + b.  A code AND-ed out of its word is the fp32
+//    denormal c * 2^(2i-149); the query carries the matching power of two,
+//    so one logic op per code and one fp32x2 FMA per two codes accumulate
+//    the exact products (no conversion step).
+//  * Values: the token weight b_t = p_t s_t (times a per-head power of two)
+//    goes through shared memory as f16; a code pair AND-ed out of its word is
+//    two f16 subnormals, each multiplied by the weight in one mixed
+//    f16 x f16 -> fp32 FMA; sum_t p_t z_t stays in fp32.  Lanes own channels.
 //  * Softmax is online in fp32 in the log2 domain (the query carries
 //    log2(e)/sqrt(D)); the running max is only raised when a score exceeds it
 //    by more than 8, which keeps all rescaling rare.
@@ -30,7 +32,10 @@
 //    the fp32 output.
 //  * Pre-RoPE caches dequantize keys explicitly and rotate them at their
 //    absolute positions (KIVI article, paragraph 4; KVQuant summary,
-//    "Pre-RoPE Key Quantization").
+//    "Pre-RoPE Key Quantization"), sin/cos from an exact Cody-Waite angle
+//    reduction and the hardware sine/cosine.
+//  * With kivi_append_decode the residual slice that holds the appended
+//    token takes it from the caller's k_t/v_t and stores it to the residual.
 #include <cuda_runtime.h>
 
 #include "kivi_common.cuh"
@@ -161,8 +166,8 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
 // 2^23 (`magic`, a runtime register so that the mask stays an immediate) gives
 // 2^23 + c*2^(2i) exactly; adding `neg` = (-2^23, -2^23) leaves
 // (c_first 2^(2i), c_second 2^(2i)).  One logic op per code; the power of two
-// is folded into the multipliers (q' for keys, p' and a per-channel-pair
-// factor for values).
+// is folded into the scales (the pre-RoPE key path uses this conversion,
+// since it dequantizes explicitly).
 __device__ __forceinline__ float2 code_pair(uint32_t w, uint32_t w16, int i, uint32_t magic,
                                             float2 neg)
 {
