@@ -173,6 +173,9 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 constexpr int kQuantThreads = 256;
+#ifndef KIVI_QUANT_CTAS
+#define KIVI_QUANT_CTAS 4   // resident CTAs per SM (persistent grid; measured best)
+#endif
 
 // The CTA works as two independent halves: threads [0, D) take the key tile,
 // the rest the value tile, each with its own named barrier (ids 1 and 2), so
@@ -378,7 +381,7 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
 }
 
 template <int D, int DT>
-__global__ void __launch_bounds__(kQuantThreads, 3) quant_kernel(QuantParams p)
+__global__ void __launch_bounds__(kQuantThreads, KIVI_QUANT_CTAS) quant_kernel(QuantParams p)
 {
     using S = QuantSmem<D>;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -477,7 +480,7 @@ static cudaError_t launch_quant_t(const QuantParams &p, cudaStream_t st)
     }
     const long long items = p.seqs * (long long)p.n_g + (p.r_copy > 0 ? p.seqs : 0);
     if (items == 0) return cudaSuccess;
-    long long grid = (long long)num_sms() * 3;
+    long long grid = (long long)num_sms() * KIVI_QUANT_CTAS;
     if (grid > items) grid = items;
     QuantParams q = p;
     q.div_ng = make_magic((unsigned long long)(p.n_g > 0 ? p.n_g : 1));
