@@ -313,6 +313,112 @@ void oracle_decode_seq(const uint16_t *q, int HG, int D, int G, int R, int dtype
     }
 }
 
+/* ---- diagnostic grouping modes (fake quantization) ----------------------- */
+
+/*
+ * The KIVI article (paragraphs 1-3) argues by comparing groupings: keys grouped
+ * per token against per channel, values per channel against per token, and the
+ * record for Llama-2-13B contrasts a naive symmetric 2-bit per-token scheme.
+ * These functions quantize a whole [T][D] matrix under any of those groupings
+ * and return the dequantized matrix, so that errors can be compared.
+ *
+ * One group of n values x_0..x_{n-1} (fp32), at `bits` bits:
+ *   asymmetric (sym = 0), L = 2^bits - 1 levels above the zero:
+ *     zero  = fp16(min), scale = fp16(fl32(fl32(max - min) / L)), a stored zero
+ *             of either sign written as +0 (the KIVI code at bits = 2);
+ *     code  = 0 if scale == 0, else clamp(rint(fl32(fl32(x - zero)/scale)), 0, L);
+ *     x_hat = code*scale + zero rounded once to fp32.
+ *   symmetric (sym = 1), L = 2^(bits-1) - 1, bits >= 2 (the plain absmax reading
+ *   of "symmetric": no zero point, scale from the largest magnitude):
+ *     scale = fp16(fl32(max|x| / L));
+ *     code  = 0 if scale == 0, else clamp(rint(fl32(x/scale)), -(L+1), L);
+ *     x_hat = code*scale (exact in fp32).
+ * Codes are returned as int (may be NULL).
+ */
+static void fq_group(const float *x, long long stride, int n, int bits, int sym,
+                     float *xhat, int *codes)
+{
+    if (!sym) {
+        float mn = x[0], mx = x[0];
+        for (int i = 1; i < n; ++i) {
+            float v = x[(long long)i * stride];
+            if (v < mn) mn = v;
+            if (v > mx) mx = v;
+        }
+        int L = (1 << bits) - 1;
+        uint16_t sb = float_to_f16_bits((mx - mn) / (float)L);
+        uint16_t zb = float_to_f16_bits(mn);
+        if ((sb & 0x7fffu) == 0) sb = 0;
+        if ((zb & 0x7fffu) == 0) zb = 0;
+        float sf = f16_bits_to_float(sb), zf = f16_bits_to_float(zb);
+        for (int i = 0; i < n; ++i) {
+            long long at = (long long)i * stride;
+            int c = 0;
+            if (sf != 0.0f) {
+                float rr = rintf((x[at] - zf) / sf);
+                if (rr < 0.0f) rr = 0.0f;
+                if (rr > (float)L) rr = (float)L;
+                c = (int)rr;
+            }
+            xhat[at] = fmaf((float)c, sf, zf);
+            if (codes) codes[at] = c;
+        }
+    } else {
+        float amax = 0.0f;
+        for (int i = 0; i < n; ++i) {
+            float a = fabsf(x[(long long)i * stride]);
+            if (a > amax) amax = a;
+        }
+        int L = (1 << (bits - 1)) - 1;
+        uint16_t sb = float_to_f16_bits(amax / (float)L);
+        float sf = f16_bits_to_float(sb);
+        for (int i = 0; i < n; ++i) {
+            long long at = (long long)i * stride;
+            int c = 0;
+            if (sf != 0.0f) {
+                float rr = rintf(x[at] / sf);
+                if (rr < (float)(-L - 1)) rr = (float)(-L - 1);
+                if (rr > (float)L) rr = (float)L;
+                c = (int)rr;
+            }
+            xhat[at] = (float)c * sf;
+            if (codes) codes[at] = c;
+        }
+    }
+}
+
+/*
+ * Fake-quantize one row-major [T][D] fp32 matrix.  axis 0 (per channel, the
+ * KIVI key grouping): group g of channel d is tokens [gG, gG+G) of column d,
+ * T a multiple of G.  axis 1 (per token, the KIVI value grouping): group j of
+ * token t is channels [jG, jG+G) of row t, D a multiple of G.  Returns 0, or
+ * -1 for an unsupported argument.
+ */
+int oracle_fake_quant(const float *x, long long T, int D, int axis, int G, int bits,
+                      int sym, float *xhat, int *codes)
+{
+    if (G < 1 || bits < 1 || bits > 8 || (sym && bits < 2)) return -1;
+    if (axis == 0) {
+        if (T % G) return -1;
+        for (int d = 0; d < D; ++d)
+            for (long long g = 0; g < T / G; ++g) {
+                long long at = g * G * D + d;
+                fq_group(x + at, D, G, bits, sym, xhat + at, codes ? codes + at : 0);
+            }
+        return 0;
+    }
+    if (axis == 1) {
+        if (D % G) return -1;
+        for (long long t = 0; t < T; ++t)
+            for (int j = 0; j < D / G; ++j) {
+                long long at = t * D + (long long)j * G;
+                fq_group(x + at, 1, G, bits, sym, xhat + at, codes ? codes + at : 0);
+            }
+        return 0;
+    }
+    return -1;
+}
+
 /* ---- byte accounting ----------------------------------------------------- */
 
 /*
