@@ -504,6 +504,112 @@ def run_e2e(args, w, caches, Ks, Vs, steps, dev, world):
             "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": ms / n}
 
 
+DIAG_MODES = {
+    # mode: ((key axis, symmetric), (value axis, symmetric)); axis 0 = per channel
+    "kivi": ((0, False), (1, False)),
+    "k_per_token": ((1, False), (1, False)),
+    "v_per_channel": ((0, False), (0, False)),
+    "naive_symmetric": ((1, True), (1, True)),
+}
+
+
+def run_diag(args):
+    """Time kivi_fake_quant over every key and value matrix of one Llama-2-13B
+    layer cache (16 x 40 heads, 4,096 tokens, head_dim 128, bf16, heavy-tailed
+    keys) under the groupings the KIVI article compares, 2 bits.  Each launch
+    reads 2 B and writes 4 B (fp32 x_hat) per element; the inputs (1.3 GB)
+    exceed L2.  Reports per-mode launch times, achieved HBM GB/s and the
+    relative Frobenius errors ||X - X_hat|| / ||X|| from the kernel's own sums."""
+    import torch
+    import bit_asymmetric_kv_prefill_b200 as kivi
+    from bit_asymmetric_kv_prefill_b200 import synth
+    from bit_asymmetric_kv_prefill_b200 import build as kbuild
+    kbuild.build()
+    L = kivi.lib()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS["llama2_13b_cache"]
+    if args.batch:
+        w = synth.scaled(w, B=args.batch)
+    K, V = synth.prefill_inputs(w, seed=0, device=dev)
+    N, T, D = w.B * w.H_kv, w.T, w.D
+    xh = torch.empty((N, T, D), dtype=torch.float32, device=dev)
+    err = torch.empty(N, dtype=torch.float64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    dt = kivi.KIVI_BF16
+    norms = {"K": float(K.double().pow(2).sum()), "V": float(V.double().pow(2).sum())}
+    src = {"K": ctypes.c_void_p(K.data_ptr()), "V": ctypes.c_void_p(V.data_ptr())}
+    xhp, errp = ctypes.c_void_p(xh.data_ptr()), ctypes.c_void_p(err.data_ptr())
+    elems = N * T * D
+
+    def launch(which, axis, sym, values=True):
+        rc = L.kivi_fake_quant(src[which], dt, N, T, D, axis, 32, 2, int(sym),
+                               xhp if values else None, errp, sp)
+        if rc:
+            raise RuntimeError(f"kivi_fake_quant failed: {kivi.status_string(rc)}")
+
+    plan = []
+    for mode, ((ka, ks), (va, vs)) in DIAG_MODES.items():
+        plan.append((mode, "K", ka, ks, True))
+        plan.append((mode, "V", va, vs, True))
+    plan.append(("kivi_error_only", "K", 0, False, False))
+    plan.append(("kivi_error_only", "V", 1, False, False))
+    for _ in range(args.warmup):
+        for _, which, axis, sym, values in plan:
+            launch(which, axis, sym, values)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in plan] for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    clocks = ClockSampler(f"{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0")
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0e.record(stream)
+    for k in range(args.steps):
+        for i, (_, which, axis, sym, values) in enumerate(plan):
+            ev[k][i][0].record(stream)
+            launch(which, axis, sym, values)
+            ev[k][i][1].record(stream)
+    t1e.record(stream)
+    torch.cuda.synchronize(dev)
+    ck = clocks.stop()
+    ms = t0e.elapsed_time(t1e)
+    peak, peak_kind = measured_peak()
+    modes = {}
+    for i, (mode, which, axis, sym, values) in enumerate(plan):
+        us = 1e3 * sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps)) / args.steps
+        nbytes = elems * (6 if values else 2)
+        m = modes.setdefault(mode, {})
+        m[f"{which}_us"] = us
+        m[f"{which}_gbs"] = nbytes / (us / 1e6) / 1e9
+    # errors of each mode (one more untimed pass, read back)
+    for mode, ((ka, ks), (va, vs)) in DIAG_MODES.items():
+        for which, axis, sym in (("K", ka, ks), ("V", va, vs)):
+            launch(which, axis, sym, values=False)
+            modes[mode][f"{which}_rel_err"] = (float(err.sum()) / norms[which]) ** 0.5
+    launches = len(plan) * args.steps
+    dom = modes["kivi"]
+    achieved = elems * 6 / (dom["K_us"] / 1e6) / 1e9
+    print(json.dumps({
+        "metric": "fake-quant elements/s", "value": launches * elems / (ms / 1e3),
+        "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+        "config": {"workload": "llama2_13b_layer_cache fake quantization, 4 groupings + error-only",
+                   "batch": w.B, "matrices": N, "T": T, "D": D, "G": 32, "bits": 2, "input": "bf16",
+                   "l2": f"inputs {2 * K.numel() * 2 / 1e9:.2f} GB vs 0.126 GB L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "kernel": "fq_channel_kernel (kivi_fake_quant, keys per channel)",
+                     "alg_bytes_per_launch": elems * 6},
+        "modes": modes, "gpu_launches": launches, "clocks": ck,
+    }), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -519,9 +625,13 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
     ap.add_argument("--decode-steps", dest="decode_steps", type=int, default=0,
                     help="override the workload's decode steps")
+    ap.add_argument("--diag", action="store_true",
+                    help="time the diagnostic grouping modes (kivi_fake_quant) instead")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.diag:
+        return run_diag(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)

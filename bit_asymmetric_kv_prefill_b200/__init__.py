@@ -11,6 +11,9 @@ calls raise if the library is missing.
     cache.prefill(K, V)              # K, V [B, H_kv, T, D] on the GPU
     cache.append(k_t, v_t)           # [B, H_kv, D]
     out = cache.decode(q)            # q [B, H_q, D] -> fp32 [B, H_q, D]
+
+    # quantize-dequantize under another grouping (diagnostics, no cache)
+    x_hat, sq_err = fake_quant(K, AXIS_PER_TOKEN, G=32, bits=2, symmetric=True)
 """
 from __future__ import annotations
 
@@ -26,6 +29,7 @@ LIB_PATH = os.environ.get("KIVI_LIB") or os.path.join(_HERE, "libkivi_b200.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "kivi.h")
 
 KIVI_F16, KIVI_BF16 = 0, 1
+AXIS_PER_CHANNEL, AXIS_PER_TOKEN = 0, 1
 STATUS = {0: "KIVI_OK", 1: "KIVI_ERR_ARG", 2: "KIVI_ERR_UNSUPPORTED", 3: "KIVI_ERR_CAPACITY",
           4: "KIVI_ERR_STATE", 5: "KIVI_ERR_OOM", 6: "KIVI_ERR_CUDA", 7: "KIVI_ERR_DEVICE"}
 
@@ -81,12 +85,13 @@ def lib():
     L.kivi_device_status.argtypes = [vp, P(i32)]
     L.kivi_cache_destroy.argtypes = [vp]
     L.kivi_decode_split.argtypes = [i64, i64, i32, i32, i32, i64, i64, i64, P(i64)]
+    L.kivi_fake_quant.argtypes = [vp, i32, i64, i64, i32, i32, i32, i32, i32, vp, vp, vp]
     for name in ("kivi_cache_create", "kivi_cache_create_ex", "kivi_cache_required_bytes",
                  "kivi_prefill", "kivi_append", "kivi_decode_attn", "kivi_decode_attn_noalloc",
                  "kivi_append_decode",
                  "kivi_cache_reset",
                  "kivi_cache_length", "kivi_cache_bytes", "kivi_export", "kivi_device_status",
-                 "kivi_cache_destroy", "kivi_decode_split"):
+                 "kivi_cache_destroy", "kivi_decode_split", "kivi_fake_quant"):
         getattr(L, name).restype = st
     _lib = L
     return L
@@ -276,3 +281,36 @@ class KiviCache:
             self.close()
         except Exception:
             pass
+
+
+def fake_quant(x: torch.Tensor, axis: int, G: int = 32, bits: int = 2, symmetric: bool = False,
+               out: torch.Tensor | None = None, error: bool = True, values: bool = True,
+               stream=None):
+    """Quantize-dequantize every [T, D] matrix of x ([..., T, D], bf16 or fp16,
+    on the GPU) under one grouping (see kivi_fake_quant): ``axis`` is
+    AXIS_PER_CHANNEL (groups of G tokens of a channel, the KIVI key rule) or
+    AXIS_PER_TOKEN (groups of G channels of a token, the KIVI value rule).
+
+    Returns (x_hat, sq_err): x_hat fp32 with x's shape (None unless
+    ``values``), sq_err fp64 [prod(leading dims)] holding sum (x - x_hat)^2 per
+    matrix (None unless ``error``)."""
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor")
+    if x.dim() < 2:
+        raise ValueError("x must have shape [..., T, D]")
+    T, D = x.shape[-2], x.shape[-1]
+    N = x.numel() // max(T * D, 1)
+    xh = None
+    if values:
+        if out is None:
+            out = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+        elif (out.dtype != torch.float32 or out.shape != x.shape or not out.is_contiguous()
+              or not out.is_cuda):
+            raise ValueError("out must be a contiguous CUDA float32 tensor shaped like x")
+        xh = out
+    err = torch.empty(N, dtype=torch.float64, device=x.device) if error else None
+    _check(lib().kivi_fake_quant(x.data_ptr(), _dtype_code(x.dtype), N, T, D, axis, G, bits,
+                                 int(symmetric), xh.data_ptr() if xh is not None else None,
+                                 err.data_ptr() if err is not None else None, _stream_ptr(stream)),
+           "kivi_fake_quant")
+    return xh, err

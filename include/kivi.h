@@ -214,6 +214,47 @@ KIVI_API kivi_status kivi_decode_split(long long seqs, long long n_groups, int r
                               long long warps, long long seq, long long warp,
                               long long out[4]);
 
+/*
+ * Diagnostic quantization under the groupings the KIVI article compares
+ * ("KIVI Quantization Secures Llama-2 Accuracy at Two Bits", paragraphs 2-3:
+ * keys and values grouped per token or per channel; record
+ * kv-efficiency/kivi-2bit-llama2-13b-mha-4k, "Quality": the naive symmetric
+ * per-token 2-bit baseline).  It quantizes and dequantizes N independent
+ * [T, D] matrices and reports the result and its squared error; it does not
+ * touch any cache.
+ *
+ *   x       DEVICE [N, T, D] in `dtype`, 16-byte aligned, caller-owned.
+ *   axis    KIVI_AXIS_PER_CHANNEL: group g of channel d is tokens [gG, gG+G)
+ *           of column d (the KIVI key grouping; T % G == 0, any G >= 1);
+ *           KIVI_AXIS_PER_TOKEN: group j of token t is channels [jG, jG+G) of
+ *           row t (the KIVI value grouping; D % G == 0, G a power of two in
+ *           [8, 256], else KIVI_ERR_UNSUPPORTED).
+ *   bits    1..8 (asymmetric) or 2..8 (symmetric).
+ *   symmetric = 0: zero = fp16(group min), scale = fp16((max - min)/(2^bits - 1))
+ *           (subtraction and division rounded in fp32), code = clamp(rint((x -
+ *           zero)/scale), 0, 2^bits - 1) with IEEE fp32 division and rint half
+ *           to even, x_hat = code*scale + zero rounded once to fp32; at bits = 2
+ *           this is the cache's own code.  symmetric != 0 (absmax, no zero):
+ *           scale = fp16(max|x| / (2^(bits-1) - 1)), code = clamp(rint(x/scale),
+ *           -2^(bits-1), 2^(bits-1) - 1), x_hat = code*scale.  A zero scale
+ *           gives code 0.  A stored zero of either sign is +0.
+ *   xhat    DEVICE [N, T, D] fp32, 16-byte aligned, or NULL.
+ *   sq_err  DEVICE [N] fp64, 8-byte aligned, or NULL: set to the sum over each
+ *           matrix of (x - x_hat)^2.  Each difference is rounded to fp32 and
+ *           squared and summed in fp32 over runs of at most 8 elements (one
+ *           rounding per element, fused); the run sums are added in fp64 in an
+ *           unspecified order.  Relative error below 10 * 2^-24.
+ * At least one of xhat, sq_err is non-NULL; D is a multiple of 8; T*D <= 2^33
+ * (else KIVI_ERR_UNSUPPORTED).  Values whose fp16 scale or zero overflows
+ * (|x| near 65504) give non-finite results.  Asynchronous on `stream`; errors
+ * as the other calls (KIVI_ERR_ARG for bad pointers, sizes or alignment).
+ */
+typedef enum { KIVI_AXIS_PER_CHANNEL = 0, KIVI_AXIS_PER_TOKEN = 1 } kivi_axis;
+
+KIVI_API kivi_status kivi_fake_quant(const void *x, kivi_dtype dtype, long long N, long long T,
+                                     int D, int axis, int G, int bits, int symmetric,
+                                     float *xhat, double *sq_err, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

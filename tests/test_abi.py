@@ -73,6 +73,36 @@ def test_null_handles_are_rejected():
     assert L.kivi_cache_length(None, None, None) == 1
 
 
+# kivi_fake_quant(x, dtype, N, T, D, axis, G, bits, symmetric, xhat, sq_err, stream);
+# the pointers below are never dereferenced: every case fails its argument check.
+_FQ = dict(x=256, dtype=kivi.KIVI_BF16, N=2, T=64, D=128, axis=kivi.AXIS_PER_TOKEN, G=32,
+           bits=2, sym=0, xhat=512, err=None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=None), 1),
+    (dict(xhat=None, err=None), 1),
+    (dict(x=258), 1),                           # x not 16-byte aligned
+    (dict(xhat=520), 1),                        # x_hat not 16-byte aligned
+    (dict(err=260), 1),                         # sq_err not 8-byte aligned
+    (dict(dtype=3), 1),
+    (dict(N=0), 1), (dict(T=0), 1), (dict(D=12), 1), (dict(D=0), 1),
+    (dict(axis=2), 1),
+    (dict(bits=0), 1), (dict(bits=9), 1), (dict(bits=1, sym=1), 1),
+    (dict(G=0), 1),
+    (dict(G=48), 1),                            # per token: D % G != 0
+    (dict(axis=kivi.AXIS_PER_CHANNEL, G=48), 1),  # per channel: T % G != 0
+    (dict(G=4, D=128), 2),                      # per-token group below one vector
+    (dict(G=512, D=1024), 2),                   # per-token group wider than a warp
+    (dict(T=1 << 27, D=128), 2),                # T*D above 2^33
+])
+def test_fake_quant_rejects_bad_arguments_before_any_launch(kw, code):
+    a = dict(_FQ, **kw)
+    assert kivi.lib().kivi_fake_quant(a["x"], a["dtype"], a["N"], a["T"], a["D"], a["axis"],
+                                      a["G"], a["bits"], a["sym"], a["xhat"], a["err"],
+                                      None) == code
+
+
 @pytest.mark.parametrize("seqs,n_groups,r,wg,wr,warps", [
     (1, 4, 128, 4, 3, 26),        # tiny workload: 4 groups + 22 residual items
     (256, 128, 1, 4, 3, 2368),    # Llama-2-7B layer after the first flush
