@@ -590,6 +590,20 @@ def run_diag(args):
             launch(which, axis, sym, values=False)
             modes[mode][f"{which}_rel_err"] = (float(err.sum()) / norms[which]) ** 0.5
     launches = len(plan) * args.steps
+    cpu = None
+    if not args.no_cpu_baseline:
+        # the oracle as it stands, single-threaded, on whole key matrices of
+        # the same cache (keys per channel, 2 bits), for about cpu_seconds
+        import oracle
+        Kh = K.reshape(N, T, D)
+        done, t0 = 0, time.perf_counter()
+        while done < N and (done == 0 or time.perf_counter() - t0 < args.cpu_seconds):
+            oracle.fake_quant(Kh[done].float().cpu().numpy(), 0, 32, 2, False)
+            done += 1
+        secs = time.perf_counter() - t0
+        cpu = {"value": done * T * D / secs, "unit": "elements/s", "cores": 1, "kind": "oracle",
+               "sample": f"{done} key matrices ({T} x {D}) of the same cache, per channel, "
+                         f"{secs:.1f} s single-threaded"}
     dom = modes["kivi"]
     achieved = elems * 6 / (dom["K_us"] / 1e6) / 1e9
     print(json.dumps({
@@ -605,7 +619,7 @@ def run_diag(args):
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                      "kernel": "fq_channel_kernel (kivi_fake_quant, keys per channel)",
                      "alg_bytes_per_launch": elems * 6},
-        "modes": modes, "gpu_launches": launches, "clocks": ck,
+        "modes": modes, "gpu_launches": launches, "clocks": ck, "cpu_baseline": cpu,
     }), flush=True)
     return 0
 
