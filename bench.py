@@ -443,7 +443,10 @@ def run_gpu(args):
                          "kernel": "decode_kernel (kivi_decode_attn)",
                          "alg_bytes_per_launch": bytes_per_launch,
                          "frac_of_8TBps": achieved / 8000.0},
-            "decode_attn": {"avg_us": 1e3 * dec_avg, "launches_timed": len(dec_ms),
+            "decode_attn": {"avg_us": 1e3 * dec_avg,
+                            "median_us": 1e3 * statistics.median(dec_ms),
+                            "p90_us": 1e3 * sorted(dec_ms)[int(0.9 * (len(dec_ms) - 1))],
+                            "launches_timed": len(dec_ms),
                             "tokens_heads_per_s": units_step / nl / w.steps / (dec_avg / 1e3),
                             "gpu_time_share": sum(dec_ms) / ms_local},
             "e2e": e2e, "gpu_launches": launches_step * args.steps, "clocks": ck,
