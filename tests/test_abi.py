@@ -62,6 +62,19 @@ def test_bad_configs_are_rejected_before_any_launch(kw, code):
     assert kivi.lib().kivi_cache_required_bytes(ctypes.byref(cfg), ctypes.byref(n)) == code
 
 
+def test_pre_rope_length_limit():
+    """Pre-RoPE caches hold at most 823,000 tokens (the decode's exact angle
+    reduction); plain caches have no such limit."""
+    n = ctypes.c_size_t()
+    L = kivi.lib()
+    ok = _cfg(pre_rope=1, T_max=823000)
+    assert L.kivi_cache_required_bytes(ctypes.byref(ok), ctypes.byref(n)) == 0 and n.value > 0
+    over = _cfg(pre_rope=1, T_max=823001)
+    assert L.kivi_cache_required_bytes(ctypes.byref(over), ctypes.byref(n)) == 2
+    plain = _cfg(pre_rope=0, T_max=4000000)
+    assert L.kivi_cache_required_bytes(ctypes.byref(plain), ctypes.byref(n)) == 0
+
+
 def test_null_handles_are_rejected():
     L = kivi.lib()
     assert L.kivi_prefill(None, None, None, 10, None) == 1

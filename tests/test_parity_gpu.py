@@ -110,6 +110,20 @@ def test_pre_rope_small(kw):
     run_stream(w, seed=4, steps=w.steps)
 
 
+def test_pre_rope_eight_heads_per_kv_head_and_head_dim_64():
+    w = small("long_context", B=2, H_q=16, H_kv=2, T=300, steps=12)
+    run_stream(w, seed=7, steps=w.steps)
+    w = small("tiny", B=2, H_q=4, H_kv=2, T=333, steps=6, pre_rope=True)
+    run_stream(w, seed=8, steps=w.steps)
+
+
+def test_pre_rope_longest_supported_context():
+    """A pre-RoPE cache near its 823,000-token limit (822,000 prefill tokens and
+    one append): the largest RoPE angles the decode's exact reduction serves."""
+    w = small("long_context", B=1, H_q=1, H_kv=1, T=822000, steps=1)
+    run_stream(w, seed=6, steps=1)
+
+
 def test_head_dim_64_bf16_and_128_fp16():
     run_stream(small("tiny", dtype="bf16", T=400, B=2, steps=10), seed=5, steps=10)
     run_stream(small("llama2_7b_layer", dtype="fp16", T=400, B=1, H_q=2, H_kv=2, steps=10),
