@@ -68,7 +68,7 @@ def lib():
     L.oracle_rope_inv_freq.argtypes = [c_int, c_d, f32p]
     L.oracle_rope_row.argtypes = [f64p, c_int, c_ll, f32p]
     L.oracle_kv_bytes.argtypes = [c_ll, c_ll, c_ll, c_ll, c_ll, c_int, c_int, c_ll, f64p]
-    L.oracle_fake_quant.argtypes = [f32p, c_ll, c_int, c_int, c_int, c_int, c_int, f32p, i32p]
+    L.oracle_fake_quant.argtypes = [f32p, c_ll, c_int, c_int, c_int, c_int, c_int, c_int, f32p, i32p]
     L.oracle_bf16_to_float.argtypes = [ctypes.c_uint16]
     L.oracle_bf16_to_float.restype = ctypes.c_float
     L.oracle_f16_to_float.argtypes = [ctypes.c_uint16]
@@ -138,11 +138,15 @@ AXIS_PER_CHANNEL = 0   # groups of G consecutive tokens of one channel (KIVI key
 AXIS_PER_TOKEN = 1     # groups of G consecutive channels of one token (KIVI values)
 
 
+OUTLIER_CODE = -1000   # code reported for a group's sparse (exactly kept) element
+
+
 def fake_quant(x: np.ndarray, axis: int, G: int = 32, bits: int = 2, sym: bool = False,
-               codes: bool = False):
+               codes: bool = False, outlier: int = 0):
     """Quantize-dequantize every [T, D] matrix of x (fp32, shape [..., T, D])
-    under one grouping (see oracle_fake_quant).  Returns x_hat (fp32, same
-    shape), and the integer codes too when ``codes``."""
+    under one grouping (see oracle_fake_quant); ``outlier`` = 1 keeps each
+    group's largest-magnitude element exactly (dense-and-sparse).  Returns
+    x_hat (fp32, same shape), and the integer codes too when ``codes``."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     T, D = x.shape[-2:]
     flat = x.reshape(-1, T, D)
@@ -154,11 +158,11 @@ def fake_quant(x: np.ndarray, axis: int, G: int = 32, bits: int = 2, sym: bool =
         oi = np.zeros((T, D), np.float32)
         ci = np.zeros((T, D), np.int32) if codes else None
         rc = L.oracle_fake_quant(_ptr(xi, ctypes.c_float), T, D, axis, G, bits, int(sym),
-                                 _ptr(oi, ctypes.c_float),
+                                 int(outlier), _ptr(oi, ctypes.c_float),
                                  _ptr(ci, ctypes.c_int) if codes else None)
         if rc != 0:
             raise ValueError(f"unsupported fake_quant arguments: T={T} D={D} axis={axis} "
-                             f"G={G} bits={bits} sym={sym}")
+                             f"G={G} bits={bits} sym={sym} outlier={outlier}")
         xh[i] = oi
         if codes:
             cc[i] = ci

@@ -22,6 +22,10 @@ reading.  The modes:
   v_per_channel    keys and values per channel, asymmetric
   naive_symmetric  keys and values per token, symmetric absmax (the record
                    kv-efficiency/kivi-2bit-llama2-13b-mha-4k, "Quality" field)
+  kivi_sparse      KIVI's grouping, each group dense-and-sparse: its largest-
+                   magnitude element kept exactly (KVQuant summary, "Per-Vector
+                   Dense-and-Sparse Quantization")
+  k_per_token_sparse  keys and values per token, dense-and-sparse
 
 and, for keys stored before or after RoPE (KVQuant summary, "Pre-RoPE Key
 Quantization"; KIVI article, paragraph 4), ``rope="pre"`` quantizes K and
@@ -36,11 +40,14 @@ import numpy as np
 
 from . import AXIS_PER_CHANNEL, AXIS_PER_TOKEN, fake_quant, rope_row
 
+# mode: ((key axis, symmetric, sparse elements), (value axis, symmetric, sparse))
 MODES = {
-    "kivi": ((AXIS_PER_CHANNEL, False), (AXIS_PER_TOKEN, False)),
-    "k_per_token": ((AXIS_PER_TOKEN, False), (AXIS_PER_TOKEN, False)),
-    "v_per_channel": ((AXIS_PER_CHANNEL, False), (AXIS_PER_CHANNEL, False)),
-    "naive_symmetric": ((AXIS_PER_TOKEN, True), (AXIS_PER_TOKEN, True)),
+    "kivi": ((AXIS_PER_CHANNEL, False, 0), (AXIS_PER_TOKEN, False, 0)),
+    "k_per_token": ((AXIS_PER_TOKEN, False, 0), (AXIS_PER_TOKEN, False, 0)),
+    "v_per_channel": ((AXIS_PER_CHANNEL, False, 0), (AXIS_PER_CHANNEL, False, 0)),
+    "naive_symmetric": ((AXIS_PER_TOKEN, True, 0), (AXIS_PER_TOKEN, True, 0)),
+    "kivi_sparse": ((AXIS_PER_CHANNEL, False, 1), (AXIS_PER_TOKEN, False, 1)),
+    "k_per_token_sparse": ((AXIS_PER_TOKEN, False, 1), (AXIS_PER_TOKEN, False, 1)),
 }
 
 
@@ -70,21 +77,21 @@ def errors(K: np.ndarray, V: np.ndarray, q: np.ndarray, mode: str = "kivi", G: i
            bits: int = 2, rope: str | None = None, theta: float = 10000.0) -> dict:
     """Errors of one mode.  K, V: exact fp32 values [H, T, D] (keys before RoPE
     when ``rope`` is given); q: [H, M, D] queries (after RoPE)."""
-    (ka, ks), (va, vs) = MODES[mode]
+    (ka, ks, ko), (va, vs, vo) = MODES[mode]
     K = np.asarray(K, np.float32)
     V = np.asarray(V, np.float32)
     if rope is None:
         K_ref = K.astype(np.float64)
-        K_hat = fake_quant(K, ka, G, bits, ks).astype(np.float64)
+        K_hat = fake_quant(K, ka, G, bits, ks, outlier=ko).astype(np.float64)
     elif rope == "pre":
         K_ref = rotate(K, theta)
-        K_hat = rotate(fake_quant(K, ka, G, bits, ks), theta)
+        K_hat = rotate(fake_quant(K, ka, G, bits, ks, outlier=ko), theta)
     elif rope == "post":
         K_ref = rotate(K, theta)
-        K_hat = fake_quant(K_ref.astype(np.float32), ka, G, bits, ks).astype(np.float64)
+        K_hat = fake_quant(K_ref.astype(np.float32), ka, G, bits, ks, outlier=ko).astype(np.float64)
     else:
         raise ValueError(f"rope must be None, 'pre' or 'post', got {rope!r}")
-    V_hat = fake_quant(V, va, G, bits, vs).astype(np.float64)
+    V_hat = fake_quant(V, va, G, bits, vs, outlier=vo).astype(np.float64)
     V_ref = V.astype(np.float64)
     o = attention(q, K_ref, V_ref)
     o_hat = attention(q, K_hat, V_hat)

@@ -333,14 +333,32 @@ void oracle_decode_seq(const uint16_t *q, int HG, int D, int G, int R, int dtype
  *     scale = fp16(fl32(max|x| / L));
  *     code  = 0 if scale == 0, else clamp(rint(fl32(x/scale)), -(L+1), L);
  *     x_hat = code*scale (exact in fp32).
+ * With outlier = 1 the group is split dense-and-sparse (KVQuant summary,
+ * "Per-Vector Dense-and-Sparse Quantization"): its element of largest |x| (the
+ * first one on ties) is kept exactly, x_hat = x, reported with code
+ * FQ_OUTLIER_CODE, and the other n - 1 elements are quantized as above with the
+ * statistics (min, max or max|x|) taken over them alone.
  * Codes are returned as int (may be NULL).
  */
-static void fq_group(const float *x, long long stride, int n, int bits, int sym,
+#define FQ_OUTLIER_CODE (-1000)
+
+static void fq_group(const float *x, long long stride, int n, int bits, int sym, int outlier,
                      float *xhat, int *codes)
 {
+    int o = -1; /* the sparse element, if any */
+    if (outlier) {
+        o = 0;
+        for (int i = 1; i < n; ++i)
+            if (fabsf(x[(long long)i * stride]) > fabsf(x[(long long)o * stride])) o = i;
+        xhat[(long long)o * stride] = x[(long long)o * stride];
+        if (codes) codes[(long long)o * stride] = FQ_OUTLIER_CODE;
+        if (n == 1) return;
+    }
+    int first = o == 0 ? 1 : 0; /* first dense element */
     if (!sym) {
-        float mn = x[0], mx = x[0];
-        for (int i = 1; i < n; ++i) {
+        float mn = x[(long long)first * stride], mx = mn;
+        for (int i = first + 1; i < n; ++i) {
+            if (i == o) continue;
             float v = x[(long long)i * stride];
             if (v < mn) mn = v;
             if (v > mx) mx = v;
@@ -352,6 +370,7 @@ static void fq_group(const float *x, long long stride, int n, int bits, int sym,
         if ((zb & 0x7fffu) == 0) zb = 0;
         float sf = f16_bits_to_float(sb), zf = f16_bits_to_float(zb);
         for (int i = 0; i < n; ++i) {
+            if (i == o) continue;
             long long at = (long long)i * stride;
             int c = 0;
             if (sf != 0.0f) {
@@ -366,6 +385,7 @@ static void fq_group(const float *x, long long stride, int n, int bits, int sym,
     } else {
         float amax = 0.0f;
         for (int i = 0; i < n; ++i) {
+            if (i == o) continue;
             float a = fabsf(x[(long long)i * stride]);
             if (a > amax) amax = a;
         }
@@ -373,6 +393,7 @@ static void fq_group(const float *x, long long stride, int n, int bits, int sym,
         uint16_t sb = float_to_f16_bits(amax / (float)L);
         float sf = f16_bits_to_float(sb);
         for (int i = 0; i < n; ++i) {
+            if (i == o) continue;
             long long at = (long long)i * stride;
             int c = 0;
             if (sf != 0.0f) {
@@ -391,19 +412,20 @@ static void fq_group(const float *x, long long stride, int n, int bits, int sym,
  * Fake-quantize one row-major [T][D] fp32 matrix.  axis 0 (per channel, the
  * KIVI key grouping): group g of channel d is tokens [gG, gG+G) of column d,
  * T a multiple of G.  axis 1 (per token, the KIVI value grouping): group j of
- * token t is channels [jG, jG+G) of row t, D a multiple of G.  Returns 0, or
- * -1 for an unsupported argument.
+ * token t is channels [jG, jG+G) of row t, D a multiple of G.  outlier: 0 or 1
+ * sparse elements per group.  Returns 0, or -1 for an unsupported argument.
  */
 int oracle_fake_quant(const float *x, long long T, int D, int axis, int G, int bits,
-                      int sym, float *xhat, int *codes)
+                      int sym, int outlier, float *xhat, int *codes)
 {
     if (G < 1 || bits < 1 || bits > 8 || (sym && bits < 2)) return -1;
+    if (outlier != 0 && outlier != 1) return -1;
     if (axis == 0) {
         if (T % G) return -1;
         for (int d = 0; d < D; ++d)
             for (long long g = 0; g < T / G; ++g) {
                 long long at = g * G * D + d;
-                fq_group(x + at, D, G, bits, sym, xhat + at, codes ? codes + at : 0);
+                fq_group(x + at, D, G, bits, sym, outlier, xhat + at, codes ? codes + at : 0);
             }
         return 0;
     }
@@ -412,7 +434,7 @@ int oracle_fake_quant(const float *x, long long T, int D, int axis, int G, int b
         for (long long t = 0; t < T; ++t)
             for (int j = 0; j < D / G; ++j) {
                 long long at = t * D + (long long)j * G;
-                fq_group(x + at, 1, G, bits, sym, xhat + at, codes ? codes + at : 0);
+                fq_group(x + at, 1, G, bits, sym, outlier, xhat + at, codes ? codes + at : 0);
             }
         return 0;
     }

@@ -245,3 +245,65 @@ def test_pre_rope_keys_reconstruct_better_than_post_rope():
     pre = diag.errors(K, V, q, "kivi", rope="pre")
     post = diag.errors(K, V, q, "kivi", rope="post")
     assert pre["key"] < post["key"]
+
+
+# ---- dense-and-sparse: one exactly kept element per group ----------------------
+
+@pytest.mark.parametrize("sym,bits", [(False, 2), (False, 4), (True, 2), (True, 3)])
+def test_outlier_mode_is_the_plain_code_without_that_element(sym, bits):
+    """KVQuant summary, "Per-Vector Dense-and-Sparse Quantization": the group's
+    largest-magnitude element is kept exactly and the rest is quantized as a
+    group of its own; checked against the plain mode (pinned above) applied to
+    the group with that element removed."""
+    rng = np.random.default_rng(30 + bits + 10 * sym)
+    x = mixed_matrix(40, 33, seed=bits)           # rows are groups of 33
+    x[:, 5] = 0.0
+    x[3, 7] = x[3, 9] = 1e4                        # equal magnitudes: the first wins
+    x[4, 2], x[4, 30] = -7e3, 7e3
+    xh, codes = oracle.fake_quant(x, PT, 33, bits, sym, codes=True, outlier=1)
+    for t in range(x.shape[0]):
+        o = int(np.argmax(np.abs(x[t])))           # numpy takes the first maximum too
+        assert codes[t, o] == oracle.OUTLIER_CODE and xh[t, o] == x[t, o]
+        rest = np.delete(x[t], o)[None, :]
+        ref, ref_codes = oracle.fake_quant(np.ascontiguousarray(rest), PT, 32, bits, sym, codes=True)
+        np.testing.assert_array_equal(np.delete(xh[t], o), ref[0])
+        np.testing.assert_array_equal(np.delete(codes[t], o), ref_codes[0])
+    assert codes[3, 7] == oracle.OUTLIER_CODE and codes[3, 9] != oracle.OUTLIER_CODE
+    assert codes[4, 2] == oracle.OUTLIER_CODE
+
+
+def test_outlier_mode_axes_and_degenerate_groups():
+    x = mixed_matrix(64, 96, seed=77)
+    a = oracle.fake_quant(x, PC, 32, 2, outlier=1)
+    b = oracle.fake_quant(np.ascontiguousarray(x.T), PT, 32, 2, outlier=1).T
+    np.testing.assert_array_equal(a, b)
+    # one element: kept exactly; two: the smaller-magnitude one alone is a
+    # constant group (zero scale, x_hat = fp16(x))
+    np.testing.assert_array_equal(oracle.fake_quant(x, PT, 1, 2, outlier=1), x)
+    y = np.array([[3.0, 1.1], [-0.3, 9.0]], np.float32)
+    yh = oracle.fake_quant(y, PT, 2, 2, outlier=1)
+    np.testing.assert_array_equal(yh, np.array([[3.0, np.float16(1.1)], [np.float16(-0.3), 9.0]],
+                                               np.float32))
+    with pytest.raises(ValueError):
+        oracle.fake_quant(x, PT, 32, 2, outlier=2)
+
+
+def test_outlier_mode_lossless_grid_with_spikes():
+    rng = np.random.default_rng(5)
+    k = rng.integers(0, 4, (16, 64))
+    k[:, 0::32] = 0
+    k[:, 1::32] = 3
+    x = (k * 0.25 - 1.0).astype(np.float32)
+    x[:, 17] = 5e3
+    x[:, 40] = -6e3
+    np.testing.assert_array_equal(oracle.fake_quant(x, PT, 32, 2, outlier=1), x)
+
+
+def test_one_sparse_element_rescues_per_token_keys():
+    """Per-token key groups hold about one outlier channel each on the
+    fixed-outlier workloads; keeping it exactly removes most of the error of
+    the other channels."""
+    K, _, _ = _recipe("llama2_7b_layer", heads=2)
+    plain = np.linalg.norm(K - oracle.fake_quant(K, PT))
+    sparse = np.linalg.norm(K - oracle.fake_quant(K, PT, outlier=1))
+    assert sparse < 0.6 * plain
