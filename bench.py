@@ -547,11 +547,14 @@ def run_e2e(args, w, caches, Ks, Vs, steps, dev, world):
 
 
 DIAG_MODES = {
-    # mode: ((key axis, symmetric), (value axis, symmetric)); axis 0 = per channel
-    "kivi": ((0, False), (1, False)),
-    "k_per_token": ((1, False), (1, False)),
-    "v_per_channel": ((0, False), (0, False)),
-    "naive_symmetric": ((1, True), (1, True)),
+    # mode: ((key axis, symmetric, sparse), (value axis, symmetric, sparse));
+    # axis 0 = per channel, sparse 1 = one exactly kept element per group
+    "kivi": ((0, False, 0), (1, False, 0)),
+    "k_per_token": ((1, False, 0), (1, False, 0)),
+    "v_per_channel": ((0, False, 0), (0, False, 0)),
+    "naive_symmetric": ((1, True, 0), (1, True, 0)),
+    "kivi_sparse": ((0, False, 1), (1, False, 1)),
+    "k_per_token_sparse": ((1, False, 1), (1, False, 1)),
 }
 
 
@@ -585,21 +588,21 @@ def run_diag(args):
     xhp, errp = ctypes.c_void_p(xh.data_ptr()), ctypes.c_void_p(err.data_ptr())
     elems = N * T * D
 
-    def launch(which, axis, sym, values=True):
-        rc = L.kivi_fake_quant(src[which], dt, N, T, D, axis, 32, 2, int(sym),
+    def launch(which, axis, sym, sparse, values=True):
+        rc = L.kivi_fake_quant(src[which], dt, N, T, D, axis, 32, 2, int(sym), sparse,
                                xhp if values else None, errp, sp)
         if rc:
             raise RuntimeError(f"kivi_fake_quant failed: {kivi.status_string(rc)}")
 
     plan = []
-    for mode, ((ka, ks), (va, vs)) in DIAG_MODES.items():
-        plan.append((mode, "K", ka, ks, True))
-        plan.append((mode, "V", va, vs, True))
-    plan.append(("kivi_error_only", "K", 0, False, False))
-    plan.append(("kivi_error_only", "V", 1, False, False))
+    for mode, ((ka, ks, ko), (va, vs, vo)) in DIAG_MODES.items():
+        plan.append((mode, "K", ka, ks, ko, True))
+        plan.append((mode, "V", va, vs, vo, True))
+    plan.append(("kivi_error_only", "K", 0, False, 0, False))
+    plan.append(("kivi_error_only", "V", 1, False, 0, False))
     for _ in range(args.warmup):
-        for _, which, axis, sym, values in plan:
-            launch(which, axis, sym, values)
+        for _, which, axis, sym, sparse, values in plan:
+            launch(which, axis, sym, sparse, values)
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in plan] for _ in range(args.steps)]
     props = torch.cuda.get_device_properties(dev)
@@ -610,9 +613,9 @@ def run_diag(args):
     t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0e.record(stream)
     for k in range(args.steps):
-        for i, (_, which, axis, sym, values) in enumerate(plan):
+        for i, (_, which, axis, sym, sparse, values) in enumerate(plan):
             ev[k][i][0].record(stream)
-            launch(which, axis, sym, values)
+            launch(which, axis, sym, sparse, values)
             ev[k][i][1].record(stream)
     t1e.record(stream)
     torch.cuda.synchronize(dev)
@@ -620,16 +623,16 @@ def run_diag(args):
     ms = t0e.elapsed_time(t1e)
     peak, peak_kind = measured_peak()
     modes = {}
-    for i, (mode, which, axis, sym, values) in enumerate(plan):
+    for i, (mode, which, axis, sym, sparse, values) in enumerate(plan):
         us = 1e3 * sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps)) / args.steps
         nbytes = elems * (6 if values else 2)
         m = modes.setdefault(mode, {})
         m[f"{which}_us"] = us
         m[f"{which}_gbs"] = nbytes / (us / 1e6) / 1e9
     # errors of each mode (one more untimed pass, read back)
-    for mode, ((ka, ks), (va, vs)) in DIAG_MODES.items():
-        for which, axis, sym in (("K", ka, ks), ("V", va, vs)):
-            launch(which, axis, sym, values=False)
+    for mode, ((ka, ks, ko), (va, vs, vo)) in DIAG_MODES.items():
+        for which, axis, sym, sparse in (("K", ka, ks, ko), ("V", va, vs, vo)):
+            launch(which, axis, sym, sparse, values=False)
             modes[mode][f"{which}_rel_err"] = (float(err.sum()) / norms[which]) ** 0.5
     launches = len(plan) * args.steps
     cpu = None
@@ -653,7 +656,7 @@ def run_diag(args):
         "unit": "elements/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
-        "config": {"workload": "llama2_13b_layer_cache fake quantization, 4 groupings + error-only",
+        "config": {"workload": "llama2_13b_layer_cache fake quantization, 6 groupings + error-only",
                    "batch": w.B, "matrices": N, "T": T, "D": D, "G": 32, "bits": 2, "input": "bf16",
                    "l2": f"inputs {2 * K.numel() * 2 / 1e9:.2f} GB vs 0.126 GB L2"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -85,7 +85,7 @@ def lib():
     L.kivi_device_status.argtypes = [vp, P(i32)]
     L.kivi_cache_destroy.argtypes = [vp]
     L.kivi_decode_split.argtypes = [i64, i64, i32, i32, i32, i64, i64, i64, P(i64)]
-    L.kivi_fake_quant.argtypes = [vp, i32, i64, i64, i32, i32, i32, i32, i32, vp, vp, vp]
+    L.kivi_fake_quant.argtypes = [vp, i32, i64, i64, i32, i32, i32, i32, i32, i32, vp, vp, vp]
     for name in ("kivi_cache_create", "kivi_cache_create_ex", "kivi_cache_required_bytes",
                  "kivi_prefill", "kivi_append", "kivi_decode_attn", "kivi_decode_attn_noalloc",
                  "kivi_append_decode",
@@ -285,11 +285,12 @@ class KiviCache:
 
 def fake_quant(x: torch.Tensor, axis: int, G: int = 32, bits: int = 2, symmetric: bool = False,
                out: torch.Tensor | None = None, error: bool = True, values: bool = True,
-               stream=None):
+               stream=None, outlier: int = 0):
     """Quantize-dequantize every [T, D] matrix of x ([..., T, D], bf16 or fp16,
     on the GPU) under one grouping (see kivi_fake_quant): ``axis`` is
     AXIS_PER_CHANNEL (groups of G tokens of a channel, the KIVI key rule) or
-    AXIS_PER_TOKEN (groups of G channels of a token, the KIVI value rule).
+    AXIS_PER_TOKEN (groups of G channels of a token, the KIVI value rule);
+    ``outlier`` = 1 keeps each group's largest-magnitude element exactly.
 
     Returns (x_hat, sq_err): x_hat fp32 with x's shape (None unless
     ``values``), sq_err fp64 [prod(leading dims)] holding sum (x - x_hat)^2 per
@@ -310,7 +311,8 @@ def fake_quant(x: torch.Tensor, axis: int, G: int = 32, bits: int = 2, symmetric
         xh = out
     err = torch.empty(N, dtype=torch.float64, device=x.device) if error else None
     _check(lib().kivi_fake_quant(x.data_ptr(), _dtype_code(x.dtype), N, T, D, axis, G, bits,
-                                 int(symmetric), xh.data_ptr() if xh is not None else None,
+                                 int(symmetric), int(outlier),
+                                 xh.data_ptr() if xh is not None else None,
                                  err.data_ptr() if err is not None else None, _stream_ptr(stream)),
            "kivi_fake_quant")
     return xh, err

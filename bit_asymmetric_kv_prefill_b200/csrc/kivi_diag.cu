@@ -187,11 +187,13 @@ __device__ __forceinline__ void group_params(float a, float b, float L, float &s
 // for the zero code).
 //
 // With ERR, e2 gains the squared errors (x - x_hat)^2 of the NE elements, each
-// difference rounded to fp32, squared and summed in fp32 (fused).
-template <int DT, bool SYM, bool ERR, bool EXACT, int STRIDE, int NW>
+// difference rounded to fp32, squared and summed in fp32 (fused).  With OUT,
+// the elements flagged in `sparse` (bit e) are a group's exactly kept element:
+// x_hat = x, no error.
+template <int DT, bool SYM, bool ERR, bool OUT, bool EXACT, int STRIDE, int NW>
 __device__ __forceinline__ void fq_words(const uint32_t (&w)[NW], const float *s, const float *z,
                                          const float *rs, float L, float (&h)[2 * NW], float &e2,
-                                         float &near)
+                                         float &near, unsigned sparse = 0u)
 {
     constexpr int NE = 2 * NW;
     constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
@@ -216,7 +218,9 @@ __device__ __forceinline__ void fq_words(const uint32_t (&w)[NW], const float *s
             near = __fmaf_rn(fma_sat(fabsf(__fsub_rn(y, r)), 16384.0f, -8190.0f),
                              fma_sat(fabsf(__fmaf_rn(-q, s[k], d)), 0x1p126f, 0.0f), near);
         h[e] = SYM ? __fmul_rn(r, s[k]) : __fmaf_rn(r, s[k], z[k]);
-        if (ERR) {
+        const bool keep = OUT && ((sparse >> e) & 1u);
+        if (keep) h[e] = (e & 1) ? widen<DT, 1>(w[e / 2]) : widen<DT, 0>(w[e / 2]);
+        if (ERR && !keep) {
             const float df = sub_from_h<DT>(w[e / 2], e & 1, h[e]);
             e2 = __fmaf_rn(df, df, e2);
         }
@@ -240,8 +244,9 @@ __device__ __forceinline__ void store8(float *dst, const float (&h)[8])
 // ---- per token: groups of G consecutive channels of one row -----------------
 // A lane owns one 16-byte vector (8 channels) of a row; a group of G channels
 // is G/8 adjacent lanes, reduced with xor shuffles.  A vector with a quotient
-// near a rounding boundary is redone exactly.
-template <int DT, bool SYM, bool ERR>
+// near a rounding boundary is redone exactly.  With OUT the group's element of
+// largest |x| (the first on ties) is kept exactly and the statistics skip it.
+template <int DT, bool SYM, bool ERR, bool OUT>
 __global__ void __launch_bounds__(kFqThreads, 4) fq_token_kernel(const FqParams p)
 {
     const int lane = threadIdx.x & 31;
@@ -272,7 +277,42 @@ __global__ void __launch_bounds__(kFqThreads, 4) fq_token_kernel(const FqParams 
                 // Inactive lanes form whole groups (a matrix holds whole
                 // groups), so their neutral statistics reach no active group.
                 float a = inf, c = -inf;
-                if (act) {
+                unsigned sparse = 0u;
+                if (OUT) {
+                    // (largest |x|, its element index in the group), first on ties
+                    const int base = (lane % p.lpg) * 8;
+                    float xv[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        xv[i] = (i & 1) ? widen<DT, 1>(w[i / 2]) : widen<DT, 0>(w[i / 2]);
+                    float am = -1.0f;
+                    int ai = 0x7fffffff;
+                    if (act) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            if (fabsf(xv[i]) > am) {
+                                am = fabsf(xv[i]);
+                                ai = base + i;
+                            }
+                    }
+                    for (int o = 1; o < p.lpg; o <<= 1) {
+                        const float om = __shfl_xor_sync(kFull, am, o);
+                        const int oi = __shfl_xor_sync(kFull, ai, o);
+                        if (om > am || (om == am && oi < ai)) {
+                            am = om;
+                            ai = oi;
+                        }
+                    }
+                    if (act) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            if (base + i != ai) {
+                                a = fminf(a, xv[i]);
+                                c = fmaxf(c, xv[i]);
+                            }
+                        if (ai >= base && ai < base + 8) sparse = 1u << (ai - base);
+                    }
+                } else if (act) {
                     const uint32_t mn = min2<DT>(min2<DT>(w[0], w[1]), min2<DT>(w[2], w[3]));
                     const uint32_t mx = max2<DT>(max2<DT>(w[0], w[1]), max2<DT>(w[2], w[3]));
                     a = fminf(widen<DT, 0>(mn), widen<DT, 1>(mn));
@@ -285,10 +325,10 @@ __global__ void __launch_bounds__(kFqThreads, 4) fq_token_kernel(const FqParams 
                 if (!act) continue;
                 float sc, z, rs, h[8], e2 = 0.0f, near = 0.0f;
                 group_params<SYM>(a, c, p.L, sc, z, rs);
-                fq_words<DT, SYM, ERR, false, 0, 4>(w, &sc, &z, &rs, p.L, h, e2, near);
+                fq_words<DT, SYM, ERR, OUT, false, 0, 4>(w, &sc, &z, &rs, p.L, h, e2, near, sparse);
                 if (near > 0.0f) {
                     e2 = 0.0f;
-                    fq_words<DT, SYM, ERR, true, 0, 4>(w, &sc, &z, &rs, p.L, h, e2, near);
+                    fq_words<DT, SYM, ERR, OUT, true, 0, 4>(w, &sc, &z, &rs, p.L, h, e2, near, sparse);
                 }
                 if (ERR) acc += (double)e2;
                 if (xo) store8(xo + u * 8, h);
@@ -301,8 +341,11 @@ __global__ void __launch_bounds__(kFqThreads, 4) fq_token_kernel(const FqParams 
 // ---- per channel: groups of G consecutive tokens of one channel ---------------
 // A lane owns 4 adjacent channels (one 8-byte piece of a row) of one group; a
 // unit is (token group g, piece c) of one matrix, unit = g*(D/4) + c.  A row
-// with a quotient near a rounding boundary is redone exactly.
-template <int DT, bool SYM, bool ERR>
+// with a quotient near a rounding boundary is redone exactly.  With OUT each
+// channel's element of largest |x| (the first row on ties) is kept exactly; it
+// is the first occurrence of the group's maximum or minimum, so the statistics
+// of the others are the runner-up maximum or minimum.
+template <int DT, bool SYM, bool ERR, bool OUT>
 __global__ void __launch_bounds__(kFqThreads, 3) fq_channel_kernel(const FqParams p)
 {
     const int lane = threadIdx.x & 31;
@@ -323,6 +366,51 @@ __global__ void __launch_bounds__(kFqThreads, 3) fq_channel_kernel(const FqParam
             const long long row0 = n * p.T + g * p.G;
             const uint16_t *src = p.x + row0 * p.D + col;
             const uint2 first = load8(src);
+            float sc[4], z[4], rs[4];
+            int orow[4] = {-1, -1, -1, -1};
+            if (OUT) {
+                const uint32_t f[2] = {first.x, first.y};
+                float mx1[4], mx2[4], mn1[4], mn2[4];
+                int imx[4], imn[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    mx1[e] = mn1[e] = (e & 1) ? widen<DT, 1>(f[e / 2]) : widen<DT, 0>(f[e / 2]);
+                    mx2[e] = -__int_as_float(0x7f800000);
+                    mn2[e] = __int_as_float(0x7f800000);
+                    imx[e] = imn[e] = 0;
+                }
+#pragma unroll 1
+                for (int t = 1; t < p.G; ++t) {
+                    const uint2 r2 = load8(src + (long long)t * p.D);
+                    const uint32_t g2[2] = {r2.x, r2.y};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float v = (e & 1) ? widen<DT, 1>(g2[e / 2]) : widen<DT, 0>(g2[e / 2]);
+                        if (v > mx1[e]) {
+                            mx2[e] = mx1[e];
+                            mx1[e] = v;
+                            imx[e] = t;
+                        } else if (v > mx2[e]) {
+                            mx2[e] = v;
+                        }
+                        if (v < mn1[e]) {
+                            mn2[e] = mn1[e];
+                            mn1[e] = v;
+                            imn[e] = t;
+                        } else if (v < mn2[e]) {
+                            mn2[e] = v;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float am = fabsf(mx1[e]), an = fabsf(mn1[e]);
+                    orow[e] = am > an ? imx[e] : an > am ? imn[e] : min(imx[e], imn[e]);
+                    const float dmx = orow[e] == imx[e] ? mx2[e] : mx1[e];
+                    const float dmn = orow[e] == imn[e] ? mn2[e] : mn1[e];
+                    group_params<SYM>(dmn, dmx, p.L, sc[e], z[e], rs[e]);
+                }
+            } else {
             uint32_t mn[2] = {first.x, first.y}, mx[2] = {first.x, first.y};
 #pragma unroll 1
             for (int t0 = 1; t0 < p.G; t0 += kRowBatch) {
@@ -340,11 +428,11 @@ __global__ void __launch_bounds__(kFqThreads, 3) fq_channel_kernel(const FqParam
                     }
                 }
             }
-            float sc[4], z[4], rs[4];
             group_params<SYM>(widen<DT, 0>(mn[0]), widen<DT, 0>(mx[0]), p.L, sc[0], z[0], rs[0]);
             group_params<SYM>(widen<DT, 1>(mn[0]), widen<DT, 1>(mx[0]), p.L, sc[1], z[1], rs[1]);
             group_params<SYM>(widen<DT, 0>(mn[1]), widen<DT, 0>(mx[1]), p.L, sc[2], z[2], rs[2]);
             group_params<SYM>(widen<DT, 1>(mn[1]), widen<DT, 1>(mx[1]), p.L, sc[3], z[3], rs[3]);
+            }
             float *dst = p.xhat ? p.xhat + row0 * p.D + col : nullptr;
             float e2 = 0.0f;
 #pragma unroll 1
@@ -358,10 +446,17 @@ __global__ void __launch_bounds__(kFqThreads, 3) fq_channel_kernel(const FqParam
                     if (t0 + b < p.G) {
                         const uint32_t w[2] = {v[b].x, v[b].y};
                         float h[4], e2r = 0.0f, near = 0.0f;
-                        fq_words<DT, SYM, ERR, false, 1, 2>(w, sc, z, rs, p.L, h, e2r, near);
+                        unsigned sparse = 0u;
+                        if (OUT) {
+                            const int t = t0 + b;
+                            sparse = (orow[0] == t ? 1u : 0u) | (orow[1] == t ? 2u : 0u) |
+                                     (orow[2] == t ? 4u : 0u) | (orow[3] == t ? 8u : 0u);
+                        }
+                        fq_words<DT, SYM, ERR, OUT, false, 1, 2>(w, sc, z, rs, p.L, h, e2r, near, sparse);
                         if (near > 0.0f) {
                             e2r = 0.0f;
-                            fq_words<DT, SYM, ERR, true, 1, 2>(w, sc, z, rs, p.L, h, e2r, near);
+                            fq_words<DT, SYM, ERR, OUT, true, 1, 2>(w, sc, z, rs, p.L, h, e2r, near,
+                                                                    sparse);
                         }
                         if (dst)
                             *reinterpret_cast<float4 *>(dst + (long long)(t0 + b) * p.D) =
@@ -382,7 +477,7 @@ __global__ void __launch_bounds__(kFqThreads, 3) fq_channel_kernel(const FqParam
     }
 }
 
-template <int DT, bool SYM, bool ERR>
+template <int DT, bool SYM, bool ERR, bool OUT>
 cudaError_t launch_fq(int axis, const FqParams &p, cudaStream_t st)
 {
     const long long warps_per_cta = kFqThreads / 32;
@@ -390,16 +485,20 @@ cudaError_t launch_fq(int axis, const FqParams &p, cudaStream_t st)
     const long long cap = (long long)num_sms() * (2048 / kFqThreads);
     if (grid > cap) grid = cap;
     if (axis == KIVI_AXIS_PER_TOKEN)
-        fq_token_kernel<DT, SYM, ERR><<<(unsigned)grid, kFqThreads, 0, st>>>(p);
+        fq_token_kernel<DT, SYM, ERR, OUT><<<(unsigned)grid, kFqThreads, 0, st>>>(p);
     else
-        fq_channel_kernel<DT, SYM, ERR><<<(unsigned)grid, kFqThreads, 0, st>>>(p);
+        fq_channel_kernel<DT, SYM, ERR, OUT><<<(unsigned)grid, kFqThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 
 template <int DT, bool SYM>
-cudaError_t launch_fq(int axis, const FqParams &p, cudaStream_t st)
+cudaError_t launch_fq(int axis, int outlier, const FqParams &p, cudaStream_t st)
 {
-    return p.sq_err ? launch_fq<DT, SYM, true>(axis, p, st) : launch_fq<DT, SYM, false>(axis, p, st);
+    if (outlier)
+        return p.sq_err ? launch_fq<DT, SYM, true, true>(axis, p, st)
+                        : launch_fq<DT, SYM, false, true>(axis, p, st);
+    return p.sq_err ? launch_fq<DT, SYM, true, false>(axis, p, st)
+                    : launch_fq<DT, SYM, false, false>(axis, p, st);
 }
 
 }  // namespace
@@ -409,7 +508,7 @@ using namespace kivi;
 
 extern "C" kivi_status kivi_fake_quant(const void *x, kivi_dtype dtype, long long N, long long T,
                                        int D, int axis, int G, int bits, int symmetric,
-                                       float *xhat, double *sq_err, void *stream)
+                                       int outlier, float *xhat, double *sq_err, void *stream)
 {
     if (!x || (!xhat && !sq_err)) return KIVI_ERR_ARG;
     if (((uintptr_t)x & 15u) || ((uintptr_t)xhat & 15u) || ((uintptr_t)sq_err & 7u))
@@ -418,6 +517,7 @@ extern "C" kivi_status kivi_fake_quant(const void *x, kivi_dtype dtype, long lon
     if (N < 1 || T < 1 || D < 8 || D % 8 != 0 || G < 1) return KIVI_ERR_ARG;
     if (axis != KIVI_AXIS_PER_CHANNEL && axis != KIVI_AXIS_PER_TOKEN) return KIVI_ERR_ARG;
     if (bits < (symmetric ? 2 : 1) || bits > 8) return KIVI_ERR_ARG;
+    if (outlier != 0 && outlier != 1) return KIVI_ERR_ARG;
     if (axis == KIVI_AXIS_PER_CHANNEL ? T % G != 0 : D % G != 0) return KIVI_ERR_ARG;
     if (axis == KIVI_AXIS_PER_TOKEN && (G < 8 || G > 256 || (G & (G - 1)) != 0))
         return KIVI_ERR_UNSUPPORTED;
@@ -451,8 +551,10 @@ extern "C" kivi_status kivi_fake_quant(const void *x, kivi_dtype dtype, long lon
         return KIVI_ERR_CUDA;
     cudaError_t e;
     if (dtype == KIVI_BF16)
-        e = symmetric ? launch_fq<KIVI_BF16, true>(axis, p, st) : launch_fq<KIVI_BF16, false>(axis, p, st);
+        e = symmetric ? launch_fq<KIVI_BF16, true>(axis, outlier, p, st)
+                      : launch_fq<KIVI_BF16, false>(axis, outlier, p, st);
     else
-        e = symmetric ? launch_fq<KIVI_F16, true>(axis, p, st) : launch_fq<KIVI_F16, false>(axis, p, st);
+        e = symmetric ? launch_fq<KIVI_F16, true>(axis, outlier, p, st)
+                      : launch_fq<KIVI_F16, false>(axis, outlier, p, st);
     return e == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA;
 }

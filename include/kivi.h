@@ -219,7 +219,7 @@ KIVI_API kivi_status kivi_decode_split(long long seqs, long long n_groups, int r
  * ("KIVI Quantization Secures Llama-2 Accuracy at Two Bits", paragraphs 2-3:
  * keys and values grouped per token or per channel; record
  * kv-efficiency/kivi-2bit-llama2-13b-mha-4k, "Quality": the naive symmetric
- * per-token 2-bit baseline).  It quantizes and dequantizes N independent
+ * per-token 2-bit baseline), optionally dense-and-sparse.  It quantizes and dequantizes N independent
  * [T, D] matrices and reports the result and its squared error; it does not
  * touch any cache.
  *
@@ -238,6 +238,10 @@ KIVI_API kivi_status kivi_decode_split(long long seqs, long long n_groups, int r
  *           scale = fp16(max|x| / (2^(bits-1) - 1)), code = clamp(rint(x/scale),
  *           -2^(bits-1), 2^(bits-1) - 1), x_hat = code*scale.  A zero scale
  *           gives code 0.  A stored zero of either sign is +0.
+ *   outlier 0, or 1 for dense-and-sparse groups (KVQuant summary, "Per-Vector
+ *           Dense-and-Sparse Quantization"): each group's element of largest
+ *           |x| (the first on ties) is kept exactly, x_hat = x, and the group's
+ *           statistics and codes cover the other G - 1 elements only.
  *   xhat    DEVICE [N, T, D] fp32, 16-byte aligned, or NULL.
  *   sq_err  DEVICE [N] fp64, 8-byte aligned, or NULL: set to the sum over each
  *           matrix of (x - x_hat)^2.  Each difference is rounded to fp32 and
@@ -253,7 +257,7 @@ typedef enum { KIVI_AXIS_PER_CHANNEL = 0, KIVI_AXIS_PER_TOKEN = 1 } kivi_axis;
 
 KIVI_API kivi_status kivi_fake_quant(const void *x, kivi_dtype dtype, long long N, long long T,
                                      int D, int axis, int G, int bits, int symmetric,
-                                     float *xhat, double *sq_err, void *stream);
+                                     int outlier, float *xhat, double *sq_err, void *stream);
 
 #ifdef __cplusplus
 }

@@ -89,7 +89,7 @@ def test_null_handles_are_rejected():
 # kivi_fake_quant(x, dtype, N, T, D, axis, G, bits, symmetric, xhat, sq_err, stream);
 # the pointers below are never dereferenced: every case fails its argument check.
 _FQ = dict(x=256, dtype=kivi.KIVI_BF16, N=2, T=64, D=128, axis=kivi.AXIS_PER_TOKEN, G=32,
-           bits=2, sym=0, xhat=512, err=None)
+           bits=2, sym=0, outlier=0, xhat=512, err=None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -102,6 +102,7 @@ _FQ = dict(x=256, dtype=kivi.KIVI_BF16, N=2, T=64, D=128, axis=kivi.AXIS_PER_TOK
     (dict(N=0), 1), (dict(T=0), 1), (dict(D=12), 1), (dict(D=0), 1),
     (dict(axis=2), 1),
     (dict(bits=0), 1), (dict(bits=9), 1), (dict(bits=1, sym=1), 1),
+    (dict(outlier=2), 1), (dict(outlier=-1), 1),
     (dict(G=0), 1),
     (dict(G=48), 1),                            # per token: D % G != 0
     (dict(axis=kivi.AXIS_PER_CHANNEL, G=48), 1),  # per channel: T % G != 0
@@ -112,8 +113,8 @@ _FQ = dict(x=256, dtype=kivi.KIVI_BF16, N=2, T=64, D=128, axis=kivi.AXIS_PER_TOK
 def test_fake_quant_rejects_bad_arguments_before_any_launch(kw, code):
     a = dict(_FQ, **kw)
     assert kivi.lib().kivi_fake_quant(a["x"], a["dtype"], a["N"], a["T"], a["D"], a["axis"],
-                                      a["G"], a["bits"], a["sym"], a["xhat"], a["err"],
-                                      None) == code
+                                      a["G"], a["bits"], a["sym"], a["outlier"], a["xhat"],
+                                      a["err"], None) == code
 
 
 @pytest.mark.parametrize("seqs,n_groups,r,wg,wr,warps", [

@@ -27,12 +27,12 @@ PC, PT = kv.AXIS_PER_CHANNEL, kv.AXIS_PER_TOKEN
 assert (PC, PT) == (oracle.AXIS_PER_CHANNEL, oracle.AXIS_PER_TOKEN)
 
 
-def check(x, axis, G, bits, sym):
+def check(x, axis, G, bits, sym, outlier=0):
     """Run the GPU path on x (CUDA, bf16/fp16, [..., T, D]) and compare with the oracle."""
-    xh, err = kv.fake_quant(x, axis, G, bits, sym)
+    xh, err = kv.fake_quant(x, axis, G, bits, sym, outlier=outlier)
     torch.cuda.synchronize()
     xf = x.float().cpu().numpy()
-    ref = oracle.fake_quant(xf, axis, G, bits, sym)
+    ref = oracle.fake_quant(xf, axis, G, bits, sym, outlier=outlier)
     got = xh.cpu().numpy()
     assert got.view(np.uint32).shape == ref.view(np.uint32).shape
     bad = got.view(np.uint32) != ref.view(np.uint32)
@@ -109,6 +109,33 @@ def test_error_only_and_values_only():
     assert none is None and none2 is None
     torch.testing.assert_close(err2, err, rtol=1e-12, atol=0)
     assert torch.equal(xh2, xh)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("axis", [PC, PT])
+@pytest.mark.parametrize("bits,sym", [(2, False), (3, False), (2, True), (4, True)])
+def test_dense_and_sparse_match_oracle(dtype, axis, bits, sym):
+    """One exactly kept element per group; bf16/fp16 data has many ties in |x|,
+    which exercise the first-element rule across lanes and rows."""
+    K, V = recipe("llama2_7b_layer", H=3, T=352, dtype=dtype, seed=20 + bits)
+    check(K, axis, 32, bits, sym, outlier=1)
+    check(V, axis, 32, bits, sym, outlier=1)
+    H, _ = recipe("llama2_13b_cache", H=2, T=256, dtype=dtype, seed=21)
+    check(H, axis, 32, bits, sym, outlier=1)
+
+
+def test_dense_and_sparse_group_sizes_and_ties():
+    g = torch.Generator(device="cuda").manual_seed(9)
+    x = (torch.randn((3, 96, 128), generator=g, device="cuda") * 4).round().to(torch.bfloat16)
+    x[0, :, 5] = 7.0
+    x[0, :, 6] = -7.0
+    x[1, 3, :] = -9.0
+    for G in (8, 16, 64, 128):
+        check(x, PT, G, 2, False, outlier=1)
+        check(x, PT, G, 3, True, outlier=1)
+    for G in (1, 2, 3, 32, 96):
+        check(x, PC, G, 2, False, outlier=1)
+        check(x, PC, G, 2, True, outlier=1)
 
 
 def test_two_bit_modes_are_the_cache_codec():
