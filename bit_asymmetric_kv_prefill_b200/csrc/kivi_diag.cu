@@ -380,25 +380,26 @@ __global__ void __launch_bounds__(kFqThreads, 3) fq_channel_kernel(const FqParam
                     imx[e] = imn[e] = 0;
                 }
 #pragma unroll 1
-                for (int t = 1; t < p.G; ++t) {
-                    const uint2 r2 = load8(src + (long long)t * p.D);
-                    const uint32_t g2[2] = {r2.x, r2.y};
+                for (int t0 = 1; t0 < p.G; t0 += kRowBatch) {
+                    uint2 rb[kRowBatch];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float v = (e & 1) ? widen<DT, 1>(g2[e / 2]) : widen<DT, 0>(g2[e / 2]);
-                        if (v > mx1[e]) {
-                            mx2[e] = mx1[e];
-                            mx1[e] = v;
-                            imx[e] = t;
-                        } else if (v > mx2[e]) {
-                            mx2[e] = v;
-                        }
-                        if (v < mn1[e]) {
-                            mn2[e] = mn1[e];
-                            mn1[e] = v;
-                            imn[e] = t;
-                        } else if (v < mn2[e]) {
-                            mn2[e] = v;
+                    for (int b = 0; b < kRowBatch; ++b)
+                        if (t0 + b < p.G) rb[b] = load8(src + (long long)(t0 + b) * p.D);
+#pragma unroll
+                    for (int b = 0; b < kRowBatch; ++b) {
+                        if (t0 + b >= p.G) break;
+                        const int t = t0 + b;  // rows in order: first occurrences win
+                        const uint32_t g2[2] = {rb[b].x, rb[b].y};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float v = (e & 1) ? widen<DT, 1>(g2[e / 2]) : widen<DT, 0>(g2[e / 2]);
+                            const bool up = v > mx1[e], dn = v < mn1[e];
+                            mx2[e] = up ? mx1[e] : fmaxf(mx2[e], v);
+                            mx1[e] = up ? v : mx1[e];
+                            imx[e] = up ? t : imx[e];
+                            mn2[e] = dn ? mn1[e] : fminf(mn2[e], v);
+                            mn1[e] = dn ? v : mn1[e];
+                            imn[e] = dn ? t : imn[e];
                         }
                     }
                 }
