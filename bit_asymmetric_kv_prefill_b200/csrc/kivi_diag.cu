@@ -1,17 +1,21 @@
 // kivi_diag.cu -- quantize-dequantize under the groupings the KIVI pages compare
 // (kivi_fake_quant): keys per channel or per token, values per token or per
-// channel, asymmetric min/max codes or symmetric absmax codes, 1 to 8 bits.
+// channel, asymmetric min/max codes or symmetric absmax codes, 1 to 8 bits,
+// optionally dense-and-sparse (each group's largest-magnitude element kept
+// exactly).
 //
 // Sources: "KIVI Quantization Secures Llama-2 Accuracy at Two Bits",
 // paragraphs 2-3 (reconstruction and attention-output errors of per-token and
 // per-channel grouping for keys and for values); record
 // kv-efficiency/kivi-2bit-llama2-13b-mha-4k, "Quality" field (the naive
-// symmetric per-token 2-bit baseline).  At 2 bits the asymmetric groupings are
-// the KIVI codec itself (zero = group min, scale = (max - min)/3, both stored
-// as fp16, code = rint((x - zero)/scale) clamped).
+// symmetric per-token 2-bit baseline); KVQuant summary, "Per-Vector
+// Dense-and-Sparse Quantization".  At 2 bits the asymmetric groupings are the
+// KIVI codec itself (zero = group min, scale = (max - min)/3, both stored as
+// fp16, code = rint((x - zero)/scale) clamped).
 //
-// The work is elementwise with a group reduction, bound by HBM: 2 bytes read
-// and 4 written per element (2 read when only the error is asked for).
+// The work is elementwise with a group reduction and its roofline is HBM: 2
+// bytes read and 4 written per element (2 read when only the error is asked
+// for).  The division-exact code keeps it near the issue limit as well.
 //   - Per token: a lane owns one 16-byte vector (8 channels) of a row; a group
 //     of G channels is G/8 adjacent lanes, reduced with xor shuffles.
 //   - Per channel: a lane owns 4 adjacent channels of one group of G tokens;
