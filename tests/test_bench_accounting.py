@@ -1,0 +1,73 @@
+"""The benchmark's workload arithmetic on CPU: the decode schedule, the flush
+steps and the algorithmic bytes per decode call, checked against closed forms
+written out by hand for each workload (96 B per quantized (token, kv head) and
+512 B per residual token at head_dim 128 and G = 32, plus q in bf16 and out in
+fp32), and the byte accounting against the Llama-2-13B record's 128,000 B per
+token."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from bit_asymmetric_kv_prefill_b200 import synth  # noqa: E402
+
+W = synth.WORKLOADS
+
+
+def test_schedule_and_flushes_of_the_llama2_7b_layer():
+    w = W["llama2_7b_layer"]
+    sched = bench.decode_schedule(w)
+    assert len(sched) == 64
+    # prefill of 4,096 tokens leaves 3,968 quantized + 128 residual; the first
+    # append flushes, then the residual grows by one per step
+    assert sched[0] == (4096, 1) and sched[63] == (4096, 64)
+    assert bench.flush_steps(w) == [True] + [False] * 63
+
+
+def test_schedule_of_the_gqa_stream_flushes_at_steps_1_and_129():
+    w = W["mistral_gqa"]
+    flushes = [j + 1 for j, f in enumerate(bench.flush_steps(w)) if f]
+    assert flushes == [1, 129]
+    sched = bench.decode_schedule(w)
+    assert sched[127] == (32768, 128) and sched[128] == (32896, 1) and sched[255] == (32896, 128)
+
+
+@pytest.mark.parametrize("s", [1, 2, 64])
+def test_decode_bytes_llama2_7b_layer(s):
+    w = W["llama2_7b_layer"]
+    n_q, r = bench.decode_schedule(w)[s - 1]
+    assert bench.decode_bytes(w, n_q, r) == 100_663_296 + 131_072 * s + 196_608
+
+
+def test_decode_bytes_llama2_13b_layer_and_record_basis():
+    w = W["llama2_13b_cache"]
+    # one decode over the prefilled cache: 3,968 quantized tokens + 128 residual
+    assert bench.decode_bytes(w, 3968, 128) == 286_228_480
+    # codes + full residual per token at 4,096 tokens, 40 layers: the record's
+    # 102,400 + 25,600 = 128,000 B/token
+    per_layer_codes = w.B * w.H_kv * 4096 * w.D * 2 * 2 // 8
+    per_layer_res = w.B * w.H_kv * w.R * w.D * 2 * 2
+    per_token = 40 * (per_layer_codes + per_layer_res) // (w.B * 4096)
+    assert per_token == 128_000
+
+
+@pytest.mark.parametrize("n_q,r", [(32768, 1), (32768, 128), (32896, 64)])
+def test_decode_bytes_mistral_gqa(n_q, r):
+    w = W["mistral_gqa"]
+    assert bench.decode_bytes(w, n_q, r) == 49_152 * n_q + 262_144 * r + 1_572_864
+
+
+def test_decode_bytes_long_context():
+    w = W["long_context"]
+    n_q, r = bench.decode_schedule(w)[0]
+    assert (n_q, r) == (131072, 1)
+    assert bench.decode_bytes(w, n_q, r) == 100_663_296 + 4_096 * r + 24_576
+
+
+def test_units_are_kv_tokens_times_heads():
+    w = W["llama2_7b_layer"]
+    assert bench.decode_units(w, 4096, 5) == 8 * 32 * 4101
