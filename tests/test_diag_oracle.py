@@ -255,7 +255,6 @@ def test_outlier_mode_is_the_plain_code_without_that_element(sym, bits):
     largest-magnitude element is kept exactly and the rest is quantized as a
     group of its own; checked against the plain mode (pinned above) applied to
     the group with that element removed."""
-    rng = np.random.default_rng(30 + bits + 10 * sym)
     x = mixed_matrix(40, 33, seed=bits)           # rows are groups of 33
     x[:, 5] = 0.0
     x[3, 7] = x[3, 9] = 1e4                        # equal magnitudes: the first wins
