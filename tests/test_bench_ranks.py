@@ -61,3 +61,30 @@ def test_decode_schedule_and_bytes():
     assert sched[0] == (4096, 1) and sched[-1] == (4096, 64) and len(sched) == 64
     # 96 B per quantized (token, kv head) and 512 B per residual token at D=128, G=32
     assert bench.decode_bytes(w, 4096, 1) == 8 * 32 * (4096 * 96 + 512) + 8 * 32 * 128 * 6
+
+
+def _run_bench(args, **env):
+    import json
+    import subprocess
+    e = dict(os.environ, PYTHONPATH=ROOT, **env)
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True,
+                       text=True, env=e, timeout=600, cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_runs_on_rank_0_only():
+    """Under torchrun only rank 0 times the oracle and prints; other ranks exit
+    0 without work."""
+    args = ["--impl", "reference", "--workload", "tiny", "--decode-steps", "2", "--steps", "1",
+            "--warmup", "3"]
+    assert _run_bench(args, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1") == []
+    (line,) = _run_bench(args, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
