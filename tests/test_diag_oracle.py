@@ -306,3 +306,26 @@ def test_one_sparse_element_rescues_per_token_keys():
     plain = np.linalg.norm(K - oracle.fake_quant(K, PT))
     sparse = np.linalg.norm(K - oracle.fake_quant(K, PT, outlier=1))
     assert sparse < 0.6 * plain
+
+
+def test_per_token_values_win_when_attended_tokens_have_their_own_magnitude():
+    """KIVI article, paragraph 3: per-channel value groups spike the
+    attention-output error under sparse attention.  On i.i.d. values both
+    groupings tie (the workloads' values); the gap appears once tokens carry
+    their own value magnitude and attention concentrates on a few of them, as
+    in this constructed case (not one of the workloads): per-channel groups then
+    quantize a small-magnitude attended token with the scale of the others."""
+    rng = np.random.default_rng(0)
+    H, T, D, M = 2, 512, 128, 8
+    K = rng.standard_normal((H, T, D)).astype(np.float32)
+    sigma = (10.0 ** rng.uniform(-2, 0, (H, T, 1))).astype(np.float32)
+    V = (rng.standard_normal((H, T, D)) * sigma).astype(np.float32)
+    q = np.zeros((H, M, D))
+    for h in range(H):
+        for m, t in enumerate(np.argsort(sigma[h, :, 0])[:M]):
+            q[h, m] = 3.0 * K[h, t]
+    per_token = diag.errors(K, V, q, "kivi")
+    per_channel = diag.errors(K, V, q, "v_per_channel")
+    assert per_channel["attn"] > 10 * per_token["attn"]
+    # reconstruction alone does not show it as strongly
+    assert per_channel["value"] < 2 * per_token["value"]
