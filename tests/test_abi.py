@@ -199,3 +199,11 @@ def test_decode_split_matches_exact_integer_definition():
             got = tuple(kivi.decode_split(seqs, n_groups, r, wg, wr, warps, s, w))
             assert got == _split_reference(seqs, n_groups, r, wg, wr, warps, s, w), \
                 (seqs, n_groups, r, wg, wr, warps, s, w)
+
+
+def test_fake_quant_binding_rejects_host_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        kivi.fake_quant(torch.zeros(4, 64, 128, dtype=torch.bfloat16), kivi.AXIS_PER_CHANNEL)
+    with pytest.raises(ValueError):
+        kivi.fake_quant(torch.zeros(128, dtype=torch.bfloat16), kivi.AXIS_PER_TOKEN)
