@@ -173,7 +173,12 @@ def fake_quant(x: np.ndarray, axis: int, G: int = 32, bits: int = 2, sym: bool =
 # ---- the cache --------------------------------------------------------------
 
 class OracleCache:
-    """CPU model of one layer's KIVI cache for B sequences x H_kv heads."""
+    """CPU model of one layer's KIVI cache for B sequences x H_kv heads.
+
+    Each batch element b keeps its own split (nqb[b] quantized tokens, rb[b]
+    residual tokens), so a prefill may give every batch element its own
+    length; the heads of one batch element share it.  ``n_q`` and ``r`` read
+    the common split of a uniform batch."""
 
     def __init__(self, B, H_kv, D, G, R, dtype, T_max, pre_rope=False, rope_theta=10000.0):
         assert D % G == 0 and R % G == 0
@@ -191,8 +196,21 @@ class OracleCache:
         self.zV = np.zeros((B, H_kv, Tc, D // G), np.uint16)
         self.resK = np.zeros((B, H_kv, R, D), np.uint16)
         self.resV = np.zeros((B, H_kv, R, D), np.uint16)
-        self.n_q = 0
-        self.r = 0
+        self.nqb = np.zeros(B, np.int64)
+        self.rb = np.zeros(B, np.int64)
+
+    def _uniform(self, a):
+        if not (a == a[0]).all():
+            raise ValueError("the batch has per-sequence lengths; read nqb / rb")
+        return int(a[0])
+
+    @property
+    def n_q(self) -> int:
+        return self._uniform(self.nqb)
+
+    @property
+    def r(self) -> int:
+        return self._uniform(self.rb)
 
     def _seq_ptrs(self, b, h):
         U8, U16 = ctypes.c_uint8, ctypes.c_uint16
@@ -200,20 +218,26 @@ class OracleCache:
                 _ptr(self.codesV[b, h], U8), _ptr(self.sV[b, h], U16), _ptr(self.zV[b, h], U16),
                 _ptr(self.resK[b, h], U16), _ptr(self.resV[b, h], U16))
 
-    def prefill(self, K: np.ndarray, V: np.ndarray):
-        """K, V: uint16 bit patterns [B, H_kv, T, D]."""
+    def prefill(self, K: np.ndarray, V: np.ndarray, lengths=None):
+        """K, V: uint16 bit patterns [B, H_kv, T, D].  ``lengths``: optional
+        per-batch-element token counts 1 <= T_b <= T (batch element b uses
+        K[b, :, :T_b]); default T for all."""
         K = np.ascontiguousarray(K, dtype=np.uint16)
         V = np.ascontiguousarray(V, dtype=np.uint16)
         T = K.shape[2]
+        lengths = [T] * self.B if lengths is None else [int(t) for t in lengths]
+        if len(lengths) != self.B or min(lengths) < 1 or max(lengths) > T:
+            raise ValueError(f"lengths must be {self.B} values in [1, {T}], got {lengths}")
         L = lib()
         nq, r = ctypes.c_longlong(), ctypes.c_int()
         for b in range(self.B):
             for h in range(self.H):
-                kb, vb = np.ascontiguousarray(K[b, h]), np.ascontiguousarray(V[b, h])
-                L.oracle_prefill_seq(_ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16), T,
-                                     self.D, self.G, self.R, self.dtype, *self._seq_ptrs(b, h),
-                                     ctypes.byref(nq), ctypes.byref(r))
-        self.n_q, self.r = nq.value, r.value
+                kb = np.ascontiguousarray(K[b, h, :lengths[b]])
+                vb = np.ascontiguousarray(V[b, h, :lengths[b]])
+                L.oracle_prefill_seq(_ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+                                     lengths[b], self.D, self.G, self.R, self.dtype,
+                                     *self._seq_ptrs(b, h), ctypes.byref(nq), ctypes.byref(r))
+            self.nqb[b], self.rb[b] = nq.value, r.value
 
     def append(self, k: np.ndarray, v: np.ndarray):
         """k, v: uint16 bit patterns [B, H_kv, D]."""
@@ -223,12 +247,12 @@ class OracleCache:
         nq, r = ctypes.c_longlong(), ctypes.c_int()
         for b in range(self.B):
             for h in range(self.H):
-                nq.value, r.value = self.n_q, self.r
+                nq.value, r.value = int(self.nqb[b]), int(self.rb[b])
                 kb, vb = np.ascontiguousarray(k[b, h]), np.ascontiguousarray(v[b, h])
                 L.oracle_append_seq(_ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
                                     self.D, self.G, self.R, self.dtype, *self._seq_ptrs(b, h),
                                     ctypes.byref(nq), ctypes.byref(r))
-        self.n_q, self.r = nq.value, r.value
+            self.nqb[b], self.rb[b] = nq.value, r.value
 
     def decode(self, q: np.ndarray, heads=None) -> np.ndarray:
         """q: uint16 bits [B, H_q, D] -> out float32 [B, H_q, D].
@@ -239,7 +263,7 @@ class OracleCache:
         B, H_q, D = q.shape
         HG = H_q // self.H
         out = np.full((B, H_q, D), np.nan, np.float32)
-        sc = np.zeros(max(self.n_q + self.r, 1), np.float64)
+        sc = np.zeros(max(int((self.nqb + self.rb).max()), 1), np.float64)
         L = lib()
         pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(self.H)]
         for b, h in pairs:
@@ -247,7 +271,8 @@ class OracleCache:
             ob = np.zeros((HG, D), np.float32)
             L.oracle_decode_seq(_ptr(qb, ctypes.c_uint16), HG, D, self.G, self.R, self.dtype,
                                 int(self.pre_rope), self.theta, *self._seq_ptrs(b, h),
-                                self.n_q, self.r, _ptr(sc, ctypes.c_double), _ptr(ob, ctypes.c_float))
+                                int(self.nqb[b]), int(self.rb[b]), _ptr(sc, ctypes.c_double),
+                                _ptr(ob, ctypes.c_float))
             out[b, h * HG:(h + 1) * HG] = ob
         return out
 

@@ -396,3 +396,63 @@ def test_pre_rope_decode_rotates_keys_at_absolute_positions():
         Kbad[128 + i] = rope_np(from_bits(K[0, 0, 128 + i], dt), i, 10000.0)
     bad = attn_np(from_bits(q[0], dt), Kbad, from_bits(V[0, 0], dt))
     assert np.abs(bad - ref).max() > 1e-4
+
+
+# ---- per-sequence lengths in one batch ------------------------------------------
+
+def test_ragged_batch_is_independent_sequences():
+    """A batch whose elements have their own lengths (prefill T_b, then common
+    appends that flush each residual at its own step) holds, element by element,
+    exactly the store and the attention of a one-element cache of that length."""
+    w = synth.scaled(synth.WORKLOADS["tiny"], B=3, H_q=4, H_kv=2, T=300)
+    dt = oracle.DTYPE_F16
+    K, V = synth.prefill_inputs(w, seed=4)
+    kb, vb = synth.bits(K), synth.bits(V)
+    lengths = [50, 300, 129]
+    steps = 140
+    c = oracle.OracleCache(w.B, w.H_kv, w.D, w.G, w.R, dt, 300 + steps)
+    c.prefill(kb, vb, lengths=lengths)
+    singles = []
+    for b, T_b in enumerate(lengths):
+        s = oracle.OracleCache(1, w.H_kv, w.D, w.G, w.R, dt, 300 + steps)
+        s.prefill(kb[b:b + 1, :, :T_b], vb[b:b + 1, :, :T_b])
+        singles.append(s)
+    assert list(c.nqb) == [0, 256, 128] and list(c.rb) == [50, 44, 1]
+    with pytest.raises(ValueError):
+        c.n_q
+    for step in range(1, steps + 1):
+        k, v, q = (synth.bits(t) for t in synth.step_inputs(w, step, seed=4))
+        c.append(k, v)
+        for b, s in enumerate(singles):
+            s.append(k[b:b + 1], v[b:b + 1])
+        if step in (1, 78, 79, 84, 85, 127, 128, 140):
+            out = c.decode(q)
+            for b, s in enumerate(singles):
+                assert (c.nqb[b], c.rb[b]) == (s.n_q, s.r)
+                np.testing.assert_array_equal(out[b:b + 1], s.decode(q[b:b + 1]))
+    for b, s in enumerate(singles):
+        n = s.n_q
+        np.testing.assert_array_equal(c.codesK[b, :, :n], s.codesK[0, :, :n])
+        np.testing.assert_array_equal(c.sV[b, :, :n], s.sV[0, :, :n])
+        np.testing.assert_array_equal(c.resK[b, :, :s.r], s.resK[0, :, :s.r])
+
+
+def test_ragged_lossless_cache_is_textbook_attention_per_sequence():
+    dt = oracle.DTYPE_BF16
+    B, H, D, G, R = 3, 2, 64, 32, 64
+    K, V = _lossless_kv(B, H, 192, D, G, dt, 31)
+    lengths = [7, 192, 100]
+    rng = np.random.default_rng(5)
+    q = to_bits(rng.standard_normal((B, H, D)), dt)
+    c = oracle.OracleCache(B, H, D, G, R, dt, 192)
+    c.prefill(K, V, lengths=lengths)
+    out = c.decode(q)
+    for b, T_b in enumerate(lengths):
+        for h in range(H):
+            ref = attn_np(from_bits(q[b, h:h + 1], dt), from_bits(K[b, h, :T_b], dt),
+                          from_bits(V[b, h, :T_b], dt))
+            np.testing.assert_allclose(out[b, h], ref[0], rtol=1e-5, atol=1e-6)
+    with pytest.raises(ValueError):
+        c.prefill(K, V, lengths=[0, 5, 5])
+    with pytest.raises(ValueError):
+        c.prefill(K, V, lengths=[5, 193, 5])
