@@ -69,6 +69,7 @@ def lib():
     L.oracle_rope_row.argtypes = [f64p, c_int, c_ll, f32p]
     L.oracle_kv_bytes.argtypes = [c_ll, c_ll, c_ll, c_ll, c_ll, c_int, c_int, c_ll, f64p]
     L.oracle_fake_quant.argtypes = [f32p, c_ll, c_int, c_int, c_int, c_int, c_int, c_int, f32p, i32p]
+    L.oracle_fake_quant_levels.argtypes = [f32p, c_ll, c_int, c_int, c_int, c_int, f64p, f32p, i32p]
     L.oracle_bf16_to_float.argtypes = [ctypes.c_uint16]
     L.oracle_bf16_to_float.restype = ctypes.c_float
     L.oracle_f16_to_float.argtypes = [ctypes.c_uint16]
@@ -163,6 +164,34 @@ def fake_quant(x: np.ndarray, axis: int, G: int = 32, bits: int = 2, sym: bool =
         if rc != 0:
             raise ValueError(f"unsupported fake_quant arguments: T={T} D={D} axis={axis} "
                              f"G={G} bits={bits} sym={sym} outlier={outlier}")
+        xh[i] = oi
+        if codes:
+            cc[i] = ci
+    xh = xh.reshape(x.shape)
+    return (xh, cc.reshape(x.shape)) if codes else xh
+
+
+def fake_quant_levels(x: np.ndarray, axis: int, G: int, levels, codes: bool = False):
+    """Non-uniform levels (see oracle_fake_quant_levels): every group of x
+    (fp32, [..., T, D]) coded by the nearest of the normalized ``levels`` on
+    its [min, max].  Returns x_hat, and the codes too when ``codes``."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    lev = np.ascontiguousarray(levels, dtype=np.float64)
+    T, D = x.shape[-2:]
+    flat = x.reshape(-1, T, D)
+    xh = np.zeros_like(flat)
+    cc = np.zeros(flat.shape, np.int32) if codes else None
+    L = lib()
+    for i in range(flat.shape[0]):
+        xi = np.ascontiguousarray(flat[i])
+        oi = np.zeros((T, D), np.float32)
+        ci = np.zeros((T, D), np.int32) if codes else None
+        rc = L.oracle_fake_quant_levels(_ptr(xi, ctypes.c_float), T, D, axis, G, lev.size,
+                                        _ptr(lev, ctypes.c_double), _ptr(oi, ctypes.c_float),
+                                        _ptr(ci, ctypes.c_int) if codes else None)
+        if rc != 0:
+            raise ValueError(f"unsupported fake_quant_levels arguments: T={T} D={D} axis={axis} "
+                             f"G={G} levels={lev.tolist()}")
         xh[i] = oi
         if codes:
             cc[i] = ci

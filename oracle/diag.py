@@ -26,6 +26,9 @@ reading.  The modes:
                    magnitude element kept exactly (KVQuant summary, "Per-Vector
                    Dense-and-Sparse Quantization")
   k_per_token_sparse  keys and values per token, dense-and-sparse
+  kivi_nuq         KIVI's grouping with four non-uniform levels per group
+                   (KVQuant summary, "Non-Uniform KV Cache Quantization"),
+                   fitted by ``fit_levels`` to the keys and to the values
 
 and, for keys stored before or after RoPE (KVQuant summary, "Pre-RoPE Key
 Quantization"; KIVI article, paragraph 4), ``rope="pre"`` quantizes K and
@@ -38,7 +41,7 @@ import math
 
 import numpy as np
 
-from . import AXIS_PER_CHANNEL, AXIS_PER_TOKEN, fake_quant, rope_row
+from . import AXIS_PER_CHANNEL, AXIS_PER_TOKEN, fake_quant, fake_quant_levels, rope_row
 
 # mode: ((key axis, symmetric, sparse elements), (value axis, symmetric, sparse))
 MODES = {
@@ -48,7 +51,52 @@ MODES = {
     "naive_symmetric": ((AXIS_PER_TOKEN, True, 0), (AXIS_PER_TOKEN, True, 0)),
     "kivi_sparse": ((AXIS_PER_CHANNEL, False, 1), (AXIS_PER_TOKEN, False, 1)),
     "k_per_token_sparse": ((AXIS_PER_TOKEN, False, 1), (AXIS_PER_TOKEN, False, 1)),
+    "kivi_nuq": ((AXIS_PER_CHANNEL, False, "nuq"), (AXIS_PER_TOKEN, False, "nuq")),
 }
+
+
+def group_positions(x: np.ndarray, axis: int, G: int) -> np.ndarray:
+    """(x - min)/(max - min) of every element of every non-constant group
+    (float64, flattened)."""
+    x = np.asarray(x, np.float64)
+    T, D = x.shape[-2:]
+    flat = x.reshape(-1, T, D)
+    if axis == AXIS_PER_CHANNEL:
+        g = flat.reshape(flat.shape[0], T // G, G, D).transpose(0, 1, 3, 2).reshape(-1, G)
+    else:
+        g = flat.reshape(-1, G)
+    mn = g.min(axis=1, keepdims=True)
+    rg = g.max(axis=1, keepdims=True) - mn
+    keep = rg[:, 0] > 0
+    return ((g[keep] - mn[keep]) / rg[keep]).ravel()
+
+
+def fit_levels(x: np.ndarray, axis: int, G: int = 32, nlev: int = 4, iters: int = 40) -> np.ndarray:
+    """Normalized levels for ``fake_quant_levels``: Lloyd's algorithm (1-D
+    k-means) over the group positions of x, started from their nlev evenly
+    spaced quantiles (evenly spaced levels can stall with two clusters on one
+    level); each element goes to its nearest level (the lower one on ties) and
+    each level moves to the mean of its elements (a level with none stays)."""
+    u = np.sort(group_positions(x, axis, G))
+    lev = u[np.round(np.linspace(0, u.size - 1, nlev)).astype(np.int64)].copy()
+    for _ in range(iters):
+        cuts = (lev[1:] + lev[:-1]) / 2.0
+        idx = np.searchsorted(cuts, u, side="left")   # u == cut goes to the lower level
+        new = lev.copy()
+        for k in range(nlev):
+            sel = u[idx == k]
+            if sel.size:
+                new[k] = sel.mean()
+        if np.array_equal(new, lev):
+            break
+        lev = new
+    return lev
+
+
+def _quantize(x, axis, sym, sparse, G, bits):
+    if sparse == "nuq":
+        return fake_quant_levels(x, axis, G, fit_levels(x, axis, G, 1 << bits))
+    return fake_quant(x, axis, G, bits, sym, outlier=sparse)
 
 
 def rotate(K: np.ndarray, theta: float) -> np.ndarray:
@@ -82,16 +130,16 @@ def errors(K: np.ndarray, V: np.ndarray, q: np.ndarray, mode: str = "kivi", G: i
     V = np.asarray(V, np.float32)
     if rope is None:
         K_ref = K.astype(np.float64)
-        K_hat = fake_quant(K, ka, G, bits, ks, outlier=ko).astype(np.float64)
+        K_hat = _quantize(K, ka, ks, ko, G, bits).astype(np.float64)
     elif rope == "pre":
         K_ref = rotate(K, theta)
-        K_hat = rotate(fake_quant(K, ka, G, bits, ks, outlier=ko), theta)
+        K_hat = rotate(_quantize(K, ka, ks, ko, G, bits), theta)
     elif rope == "post":
         K_ref = rotate(K, theta)
-        K_hat = fake_quant(K_ref.astype(np.float32), ka, G, bits, ks, outlier=ko).astype(np.float64)
+        K_hat = _quantize(K_ref.astype(np.float32), ka, ks, ko, G, bits).astype(np.float64)
     else:
         raise ValueError(f"rope must be None, 'pre' or 'post', got {rope!r}")
-    V_hat = fake_quant(V, va, G, bits, vs, outlier=vo).astype(np.float64)
+    V_hat = _quantize(V, va, vs, vo, G, bits).astype(np.float64)
     V_ref = V.astype(np.float64)
     o = attention(q, K_ref, V_ref)
     o_hat = attention(q, K_hat, V_hat)

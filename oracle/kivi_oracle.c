@@ -441,6 +441,73 @@ int oracle_fake_quant(const float *x, long long T, int D, int axis, int G, int b
     return -1;
 }
 
+/*
+ * Non-uniform levels (KVQuant summary, "Non-Uniform KV Cache Quantization"; the
+ * pages give only the name).  Each group keeps its min and max (fp32) and
+ * codes every element by the nearest of nlev normalized levels 0 <= l_k <= 1
+ * on [min, max]: u = (x - min)/(max - min) in double, code = argmin_k
+ * |u - l_k| (the first level on ties), x_hat = fp32(min + (max - min) l_k).
+ * A constant group decodes to its value with code 0.  Same axes as
+ * oracle_fake_quant.  Returns 0, or -1 for an unsupported argument.
+ */
+static void cb_group(const float *x, long long stride, int n, int nlev, const double *lev,
+                     float *xhat, int *codes)
+{
+    float mn = x[0], mx = x[0];
+    for (int i = 1; i < n; ++i) {
+        float v = x[(long long)i * stride];
+        if (v < mn) mn = v;
+        if (v > mx) mx = v;
+    }
+    double range = (double)mx - (double)mn;
+    for (int i = 0; i < n; ++i) {
+        long long at = (long long)i * stride;
+        int c = 0;
+        if (range > 0.0) {
+            double u = ((double)x[at] - (double)mn) / range;
+            double best = fabs(u - lev[0]);
+            for (int k = 1; k < nlev; ++k) {
+                double e = fabs(u - lev[k]);
+                if (e < best) {
+                    best = e;
+                    c = k;
+                }
+            }
+            xhat[at] = (float)((double)mn + range * lev[c]);
+        } else {
+            xhat[at] = mn;
+        }
+        if (codes) codes[at] = c;
+    }
+}
+
+int oracle_fake_quant_levels(const float *x, long long T, int D, int axis, int G, int nlev,
+                             const double *levels, float *xhat, int *codes)
+{
+    if (G < 1 || nlev < 2 || nlev > 256) return -1;
+    for (int k = 0; k < nlev; ++k)
+        if (!(levels[k] >= 0.0 && levels[k] <= 1.0)) return -1;
+    if (axis == 0) {
+        if (T % G) return -1;
+        for (int d = 0; d < D; ++d)
+            for (long long g = 0; g < T / G; ++g) {
+                long long at = g * G * D + d;
+                cb_group(x + at, D, G, nlev, levels, xhat + at, codes ? codes + at : 0);
+            }
+        return 0;
+    }
+    if (axis == 1) {
+        if (D % G) return -1;
+        for (long long t = 0; t < T; ++t)
+            for (int j = 0; j < D / G; ++j) {
+                long long at = t * D + (long long)j * G;
+                cb_group(x + at, 1, G, nlev, levels, xhat + at, codes ? codes + at : 0);
+            }
+        return 0;
+    }
+    return -1;
+}
+
 /* ---- byte accounting ----------------------------------------------------- */
 
 /*

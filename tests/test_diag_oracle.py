@@ -329,3 +329,75 @@ def test_per_token_values_win_when_attended_tokens_have_their_own_magnitude():
     assert per_channel["attn"] > 10 * per_token["attn"]
     # reconstruction alone does not show it as strongly
     assert per_channel["value"] < 2 * per_token["value"]
+
+
+# ---- non-uniform levels (KVQuant's non-uniform quantization, fitted here) --------
+
+UNIFORM4 = [0.0, 1.0 / 3.0, 2.0 / 3.0, 1.0]
+
+
+def _nearest_level_ref(x, axis, G, levels):
+    """Brute force in float64: nearest level on each group's [min, max]."""
+    x64 = np.asarray(x, np.float64)
+    lev = np.asarray(levels, np.float64)
+    out = np.empty_like(x64)
+    T, D = x.shape
+    groups = ([(slice(g * G, (g + 1) * G), d) for d in range(D) for g in range(T // G)]
+              if axis == PC else [(t, slice(j * G, (j + 1) * G)) for t in range(T) for j in range(D // G)])
+    for idx in groups:
+        v = x64[idx]
+        mn, mx = v.min(), v.max()
+        if mx == mn:
+            out[idx] = mn
+            continue
+        u = (v - mn) / (mx - mn)
+        k = np.argmin(np.abs(u[:, None] - lev[None, :]), axis=1)   # first minimum on ties
+        out[idx] = mn + (mx - mn) * lev[k]
+    return out.astype(np.float32)
+
+
+@pytest.mark.parametrize("axis", [PC, PT])
+@pytest.mark.parametrize("levels", [UNIFORM4, [0.0, 0.1, 0.35, 0.9], [0.05, 0.5, 0.95],
+                                    list(np.linspace(0, 1, 16))])
+def test_levels_are_nearest_on_each_group_range(axis, levels):
+    x = mixed_matrix(64, 96, seed=len(levels) + axis)
+    xh = oracle.fake_quant_levels(x, axis, 32, levels)
+    np.testing.assert_array_equal(xh, _nearest_level_ref(x, axis, 32, levels))
+    t = oracle.fake_quant_levels(np.ascontiguousarray(x.T), 1 - axis, 32, levels).T
+    np.testing.assert_array_equal(xh, t)
+
+
+def test_levels_ties_constant_groups_and_arguments():
+    x = np.array([[0.0, 1.0, 0.25, 0.75] + [0.5] * 4, [2.0] * 8], np.float32)
+    xh, codes = oracle.fake_quant_levels(x, PT, 8, [0.0, 0.5, 1.0], codes=True)
+    assert list(codes[0, :4]) == [0, 2, 0, 1]          # 0.25 and 0.75 are ties: the lower level
+    np.testing.assert_array_equal(xh[1], x[1])
+    for bad in ([0.0, 1.5], [0.5], [-0.1, 0.5]):
+        with pytest.raises(ValueError):
+            oracle.fake_quant_levels(x, PT, 8, bad)
+
+
+def test_levels_on_their_own_grid_are_lossless_and_fitted_exactly():
+    """Groups whose elements sit at normalized positions {0, 0.2, 0.5, 1}: those
+    levels reproduce them exactly, and Lloyd's algorithm finds them."""
+    rng = np.random.default_rng(3)
+    pos = np.array([0.0, 0.2, 0.5, 1.0])
+    k = rng.integers(0, 4, (64, 64))
+    k[0::32, :] = 0
+    k[1::32, :] = 3
+    base = rng.integers(-20, 20, (2, 64)).repeat(32, axis=0)
+    x = (base + 10.0 * pos[k]).astype(np.float32)
+    np.testing.assert_array_equal(oracle.fake_quant_levels(x, PC, 32, pos), x)
+    np.testing.assert_allclose(diag.fit_levels(x, PC, 32, 4), pos, atol=1e-12)
+
+
+def test_fitted_levels_lower_the_error_of_even_levels():
+    """Lloyd's iterations never raise the squared error; on normal groups the
+    fitted four levels beat evenly spaced ones."""
+    K, V, _ = _recipe("llama2_7b_layer", heads=2, T=256)
+    for X, axis in ((K, PC), (V, PT)):
+        lev = diag.fit_levels(X, axis, 32, 4)
+        assert np.all(np.diff(lev) > 0) and lev[0] >= 0 and lev[-1] <= 1
+        fitted = np.linalg.norm(X - oracle.fake_quant_levels(X, axis, 32, lev))
+        even = np.linalg.norm(X - oracle.fake_quant_levels(X, axis, 32, UNIFORM4))
+        assert fitted < 0.95 * even
