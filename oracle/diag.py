@@ -148,3 +148,4 @@ def errors(K: np.ndarray, V: np.ndarray, q: np.ndarray, mode: str = "kivi", G: i
         value=float(np.mean([np.linalg.norm(V_ref[h] - V_hat[h]) for h in range(V.shape[0])])),
         attn=float(100.0 * np.linalg.norm(o - o_hat) / np.linalg.norm(o)),
     )
+
