@@ -82,7 +82,6 @@ kivi_status make_plan(const kivi_config *c, int sms, Plan *p)
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-kivi_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA; }
 
 // Split weights: a quantized group and a residual slice of kResTok tokens move
 // the same number of bytes (24*D); the residual slice needs far fewer
@@ -113,6 +112,18 @@ struct kivi_cache {
     bool prefilled;
     int wg, wr;
 };
+
+namespace {
+
+// Every call that touches a cache's device memory must run with the cache's
+// device current: its launches, scratch and SM count belong to that device.
+bool on_cache_device(const kivi_cache *c)
+{
+    int d = -1;
+    return cudaGetDevice(&d) == cudaSuccess && d == c->dev;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -261,6 +272,7 @@ kivi_status kivi_cache_bytes(const kivi_cache *c, kivi_bytes *out)
 kivi_status kivi_prefill(kivi_cache *c, const void *K, const void *V, long long T, void *stream)
 {
     if (!c || !K || !V || !aligned16(K) || !aligned16(V)) return KIVI_ERR_ARG;
+    if (!on_cache_device(c)) return KIVI_ERR_ARG;
     if (c->prefilled) return KIVI_ERR_STATE;
     if (T < 1) return KIVI_ERR_ARG;
     if (T > c->cfg.T_max) return KIVI_ERR_CAPACITY;
@@ -293,6 +305,7 @@ kivi_status kivi_prefill(kivi_cache *c, const void *K, const void *V, long long 
 kivi_status kivi_append(kivi_cache *c, const void *k_t, const void *v_t, void *stream)
 {
     if (!c || !k_t || !v_t || !aligned16(k_t) || !aligned16(v_t)) return KIVI_ERR_ARG;
+    if (!on_cache_device(c)) return KIVI_ERR_ARG;
     if (!c->prefilled) return KIVI_ERR_STATE;
     if (c->n_q + c->r + 1 > c->cfg.T_max) return KIVI_ERR_CAPACITY;
     const int R = c->cfg.R, D = c->cfg.D;
@@ -331,6 +344,7 @@ kivi_status kivi_append_decode(kivi_cache *c, const void *k_t, const void *v_t, 
                                int H_q, float *out, void *stream)
 {
     if (!c || !k_t || !v_t || !aligned16(k_t) || !aligned16(v_t)) return KIVI_ERR_ARG;
+    if (!on_cache_device(c)) return KIVI_ERR_ARG;
     if (!c->prefilled) return KIVI_ERR_STATE;
     if (c->n_q + c->r + 1 > c->cfg.T_max) return KIVI_ERR_CAPACITY;
     if (c->r == c->cfg.R) {   // a flush is due: the quantizer runs first
@@ -376,6 +390,7 @@ kivi_status kivi_decode_attn(kivi_cache *c, const void *q, int H_q, float *out, 
 kivi_status kivi_device_status(kivi_cache *c, int *code)
 {
     if (!c || !code) return KIVI_ERR_ARG;
+    if (!on_cache_device(c)) return KIVI_ERR_ARG;
     cudaError_t e = cudaDeviceSynchronize();
     if (e == cudaSuccess) e = cudaMemcpy(code, c->err, sizeof(int), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && *code != 0) {
@@ -517,6 +532,7 @@ kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q
                                            int *pre_rope)
 {
     if (!c || !q || !out || !p || !aligned16(q) || !aligned16(out)) return KIVI_ERR_ARG;
+    if (!on_cache_device(c)) return KIVI_ERR_ARG;
     if (!c->prefilled) return KIVI_ERR_STATE;
     if (H_q < 1 || H_q % c->cfg.H_kv != 0) return KIVI_ERR_ARG;
     const int hg = H_q / c->cfg.H_kv;

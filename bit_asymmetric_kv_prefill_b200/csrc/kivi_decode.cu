@@ -1108,15 +1108,9 @@ template <int D, int HG, int DT, bool ROPE>
 static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t st)
 {
     using S = DecodeShape<D, HG, ROPE>;
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, HG, DT, ROPE>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
-        if (e != cudaSuccess) return e;
-        configured_dev = dev;
-    }
+    static PerDeviceOnce once;
+    const cudaError_t e = set_smem_once(once, decode_kernel<D, HG, DT, ROPE>, S::SMEM);
+    if (e != cudaSuccess) return e;
     const long long grid = (p.warps + S::NW - 1) / S::NW;
     decode_kernel<D, HG, DT, ROPE><<<(unsigned)grid, S::NW * 32, S::SMEM, st>>>(p);
     return cudaGetLastError();

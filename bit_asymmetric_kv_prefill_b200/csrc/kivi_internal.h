@@ -2,6 +2,7 @@
 // kernels.  Internal to the library.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -59,6 +60,31 @@ struct DecodeParams {
 };
 
 int num_sms();
+
+// Status of a CUDA runtime result, as every entry point reports it.
+inline kivi_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA; }
+
+// A kernel's dynamic shared-memory limit belongs to each device's context, so
+// it is raised once per device.  The flags are per device and atomic: host
+// threads driving caches on different devices each configure their own; two
+// threads racing on one device both make the same (idempotent) call.
+constexpr int kMaxDevices = 64;
+struct PerDeviceOnce {
+    std::atomic<bool> done[kMaxDevices];
+};
+
+template <typename Kernel>
+cudaError_t set_smem_once(PerDeviceOnce &once, Kernel kernel, int bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (once.done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) once.done[dev].store(true, std::memory_order_release);
+    return e;
+}
 
 cudaError_t launch_quant(int D, int dtype, const QuantParams &p, cudaStream_t st);
 cudaError_t launch_append(int D, const uint16_t *k, const uint16_t *v, uint16_t *resK,

@@ -22,7 +22,7 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per device
-constexpr int kMaxDevices = 64;
+using kivi::kMaxDevices;
 
 // Tickets first, then the partials.  Shared by every call on the device.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -32,6 +32,9 @@ void *g_scratch_addr[kMaxDevices];
 
 // Device address of g_noalloc_scratch on the current device, looked up once
 // per device (the host-side symbol is only a stand-in, not a device address).
+// The address is kept for the life of the process: a cudaDeviceReset (or any
+// reset of the device's primary context) while this library is loaded
+// invalidates it, so the library must not outlive such a reset.
 cudaError_t scratch_on_current_device(void **addr)
 {
     int dev = 0;
@@ -63,14 +66,15 @@ extern "C" kivi_status kivi_decode_attn_noalloc(kivi_cache *c, const void *q, in
     const size_t part_bytes = (size_t)p.seqs * p.slots * HG * (D + 4) * sizeof(float);
     if (tick_bytes + part_bytes > kNoAllocScratchBytes) return KIVI_ERR_CAPACITY;
     void *base = nullptr;
-    if (scratch_on_current_device(&base) != cudaSuccess) {
-        cudaGetLastError();
+    cudaError_t e = scratch_on_current_device(&base);
+    if (e != cudaSuccess) {
+        cudaGetLastError();   // the lookup's error is not a launch failure: clear it
         return KIVI_ERR_CUDA;
     }
     p.tickets = (int *)base;
     p.partials = (float *)((unsigned char *)base + tick_bytes);
     // The array keeps the previous call's contents: the tickets must start at 0.
-    cudaError_t e = cudaMemsetAsync(p.tickets, 0, (size_t)p.seqs * sizeof(int), (cudaStream_t)stream);
+    e = cudaMemsetAsync(p.tickets, 0, (size_t)p.seqs * sizeof(int), (cudaStream_t)stream);
     if (e == cudaSuccess) e = kivi::launch_decode(D, HG, dtype, pre_rope, p, (cudaStream_t)stream);
-    return e == cudaSuccess ? KIVI_OK : KIVI_ERR_CUDA;
+    return kivi::cuda_status(e);
 }

@@ -469,15 +469,9 @@ template <int D, int DT>
 static cudaError_t launch_quant_t(const QuantParams &p, cudaStream_t st)
 {
     using S = QuantSmem<D>;
-    static int configured_dev = -1;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_dev != dev) {
-        cudaError_t e = cudaFuncSetAttribute(quant_kernel<D, DT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
-        if (e != cudaSuccess) return e;
-        configured_dev = dev;
-    }
+    static PerDeviceOnce once;
+    const cudaError_t e = set_smem_once(once, quant_kernel<D, DT>, S::BYTES);
+    if (e != cudaSuccess) return e;
     const long long items = p.seqs * (long long)p.n_g + (p.r_copy > 0 ? p.seqs : 0);
     if (items == 0) return cudaSuccess;
     long long grid = (long long)num_sms() * KIVI_QUANT_CTAS;

@@ -36,6 +36,10 @@
  *     was launched and the cache is unchanged.  KIVI_ERR_CUDA reports a
  *     launch or runtime failure (cudaGetLastError), after which the cache
  *     contents are undefined.
+ *   - A cache belongs to the CUDA device that was current when it was
+ *     created.  prefill, append, decode and the device-status read must be
+ *     called with that device current; otherwise they return KIVI_ERR_ARG
+ *     and launch nothing.
  *   - Sequence lengths live on the host (no device->host synchronisation in
  *     prefill, append or decode).
  *   - A cache is not thread-safe.  No call allocates device memory except
@@ -158,7 +162,8 @@ KIVI_API kivi_status kivi_append_decode(kivi_cache *c, const void *k_t, const vo
  * allocates nothing and calls no allocating routine.
  *   - The first call on a device looks up that array's device address (once
  *     per device, with the device current); make that first call before any
- *     stream capture.
+ *     stream capture.  The address is kept until the process exits, so the
+ *     library must not outlive a reset of the device (cudaDeviceReset).
  *   - Every call shares the array and it keeps the last call's contents; the
  *     call clears the tickets it needs on `stream` before its kernel.  Calls
  *     whose kernels overlap on the GPU (any caches, any streams) race on the

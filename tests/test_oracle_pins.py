@@ -68,6 +68,21 @@ def test_kv_bytes_match_printed_record():
         assert got[k] == pytest.approx(v, rel=1e-12, abs=0), k
 
 
+def test_kv_bytes_metadata_equals_the_scale_zero_entries_of_a_cache():
+    # The metadata figure (which the record leaves out) is the fp16 scale and
+    # zero of every group: count the entries an oracle cache of one layer
+    # holds for a 4,096-token capacity (keys: one pair per channel per G
+    # tokens; values: one pair per G channels per token), 2 bytes each.
+    for heads, D, G, T in ((40, 128, 32, 4096), (8, 64, 32, 1024), (3, 128, 64, 640)):
+        c = oracle.OracleCache(1, heads, D, G, 2 * G, oracle.DTYPE_BF16, T)
+        entries = c.sK.size + c.zK.size + c.sV.size + c.zV.size
+        per_token_layer = 2 * entries / T
+        for layers in (1, 40):
+            got = oracle.kv_bytes(layers, heads, D, 2 * G, T, G=G)["metadata_per_token"]
+            assert got == layers * per_token_layer
+    assert oracle.kv_bytes(40, 40, 128, 128, 4096)["metadata_per_token"] == 51200
+
+
 def test_kv_bytes_falls_toward_8x_with_context():
     # The record notes the reduction falls toward 8x only as context grows.
     r = [oracle.kv_bytes(40, 40, 128, 128, c)["reduction"] for c in (4096, 65536, 1 << 24)]

@@ -298,6 +298,28 @@ def test_errors_and_capacity():
     assert c.device_status() == 0
 
 
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs a second visible CUDA device")
+def test_calls_with_another_device_current_are_refused():
+    """A cache belongs to the device current at its creation: calls made with
+    another device current are refused before any launch."""
+    w = small("tiny", T=40, steps=0)
+    K, V = synth.prefill_inputs(w, 0, device="cuda:0")
+    k, v, q = synth.step_inputs(w, 1, 0, device="cuda:0")
+    c = KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, T_max=48)
+    c.prefill(K, V)
+    torch.cuda.set_device(1)
+    try:
+        for call in (lambda: c.append(k, v), lambda: c.decode(q), lambda: c.append_decode(k, v, q)):
+            with pytest.raises(KiviError) as e:
+                call()
+            assert e.value.code == 1
+    finally:
+        torch.cuda.set_device(0)
+    assert c.length() == (0, 40)
+    c.append(k, v)
+    assert c.length() == (0, 41) and c.device_status() == 0
+
+
 def test_caller_workspace_holds_the_whole_cache():
     w = small("tiny", T=300, B=2, steps=0)
     n = KiviCache.required_bytes(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, 300)
@@ -363,9 +385,9 @@ def test_full_llama2_13b_cache_bytes_and_two_layers():
     assert per_tok(nb["codes"]) == 102400
     assert per_tok(nb["residual"]) == 25600
     assert per_tok(nb["codes"] + nb["residual"]) == 128000
-    assert per_tok(nb["meta"]) == 51200
     ob = oracle.kv_bytes(w.layers, w.H_kv, w.D, w.R, w.T)
     assert per_tok(nb["codes"] + nb["residual"]) == ob["sum_per_token"]
+    assert per_tok(nb["meta"]) == ob["metadata_per_token"] == 51200
 
 
 def test_full_mistral_gqa():
