@@ -1,31 +1,38 @@
 """Benchmark: KIVI 2-bit KV cache hot path on B200.
 
-One step = one pass of the whole hot path over the Llama-2-7B layer workload
-(batch 8, 32 MHA heads, head_dim 128, 4,096-token context, G=32, R=128, bf16):
-prefill quantization, then 64 decode steps each appending one token (the first
-append flushes the full residual) and running decode attention, the append fused
-into the decode launch (kivi_append_decode) except where it flushes.  The step runs
-over `--layers` independent layer caches (default 8) visited round-robin, as a
-model's decode does, so the working set (~1.1 GB) is far larger than the
-126 MB L2 and every decode streams its cache from HBM.
+The reported line is the largest single-GPU workload, the GQA Mistral-7B-like
+stream: batch 64, 32 query heads over 8 kv heads, head_dim 128, a 32,768-token
+context, G=32, R=128, bf16.  One step is one pass of the whole hot path over
+it: prefill quantization of the context, then 256 decode steps, each appending
+one token (the full residual flushes at steps 1 and 129) and running decode
+attention; the append is fused into the decode launch (kivi_append_decode)
+except where it flushes.  The packed cache (1.6 GB) is far larger than the
+126 MB L2, so every decode streams it from HBM.
 
-Metric: decode-attention KV tokens x heads per second (sum over decode calls of
-B * H_kv * tokens attended), whole step time in the denominator (prefill and
-appends included).  The decode kernel's achieved HBM bandwidth (algorithmic
-bytes / CUDA-event duration of each launch) is reported against the measured
-copy bandwidth in MEASURED_PEAKS.json.
+Metric: decode-attention KV tokens x heads per second (sum over decode calls
+of B * H_kv * tokens attended), whole step time in the denominator (prefill
+and appends included).  The decode kernel's achieved HBM bandwidth
+(algorithmic bytes / CUDA-event duration of each launch) is reported against
+the measured copy bandwidth in MEASURED_PEAKS.json.
+
+`per_config` in the same line measures the other workloads the same way:
+  llama2_7b_layer   batch 8, 32 MHA heads, 4,096 tokens, prefill + 64 steps,
+                    8 layer caches visited round-robin;
+  llama2_13b_cache  40 layers of batch 16 x 40 MHA heads at 4,096 tokens:
+                    each layer's prefill and one decode over it, with the
+                    cache bytes checked against the record's 128,000 B/token;
+  long_context      batch 1, 32/8 heads, 131,072 tokens, keys pre-RoPE:
+                    the timed 128K-token prefill and 32 decode steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload NAME] [--batch B] [--decode-steps S] [--layers L]
-
-The default workload is the Llama-2-7B layer above; `--workload` times any
-other workload of synth.WORKLOADS the same way (a step being its prefill and
-decode steps), `--batch` and `--decode-steps` shrink it.
+                    [--no-per-config] [--no-cpu-baseline] [--diag]
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own replica
 (no data exchange: sequences and heads are independent) and the reported value
 is the sum over ranks divided by the slowest rank's time.  `--impl reference`
-times the plain CPU oracle on a bounded sample of the same workload.
+times the plain CPU oracle on a bounded sample of the same workload, on the
+host's cores.
 """
 from __future__ import annotations
 
@@ -47,49 +54,72 @@ if ROOT not in sys.path:
 
 METRIC = "decode-attn KV tokens·heads/s and achieved HBM GB/s vs 8 TB/s"
 UNIT = "KV tokens·heads/s"
-WORKLOAD = "llama2_7b_layer"
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "decode_llama2_7b_layer_traffic.json")
+WORKLOAD = "mistral_gqa"
+PER_CONFIG = ("llama2_7b_layer", "llama2_13b_cache", "long_context")
+WORKLOAD_NAMES = ["tiny", "llama2_7b_layer", "llama2_13b_cache", "mistral_gqa", "long_context"]
+# Layer caches per step (visited round-robin) and distinct prefill inputs they
+# share: the Llama-2-13B cache has 40 layers; four input sets keep its inputs
+# at 11 GB while every layer keeps its own cache.
+LAYERS = {"tiny": 8, "llama2_7b_layer": 8, "llama2_13b_cache": 40, "mistral_gqa": 1,
+          "long_context": 8}
+INPUT_SETS = {"llama2_13b_cache": 4}
+# Decode steps per sequence the CPU oracle runs in its bounded sample.
+ORACLE_STEPS = {"mistral_gqa": 8, "long_context": 2}
+PROFILE_TRAFFIC = {
+    "llama2_7b_layer": os.path.join(ROOT, "profiles", "decode_llama2_7b_layer_traffic.json"),
+    "mistral_gqa": os.path.join(ROOT, "profiles", "decode_mistral_gqa_traffic.json"),
+}
 DECODE_SOURCES = ["bit_asymmetric_kv_prefill_b200/csrc/kivi_decode.cu",
                   "bit_asymmetric_kv_prefill_b200/csrc/kivi_common.cuh"]
 
 
 # ---- workload arithmetic (bytes and units, no method math) ---------------------
 
-def decode_schedule(w):
-    """(n_q, r) seen by each decode call of one layer's step, in order."""
+def decode_calls(w):
+    """Decode calls of one layer's step, in order: (n_q, r, kind) seen by each,
+    kind "flush" (its append quantizes the full residual first, a separate
+    launch), "fused" (append fused into the decode launch) or "none" (a
+    workload without decode steps: one decode over the prefilled cache)."""
     R, T = w.R, w.T
     n_q = R * ((T - 1) // R)
     r = T - n_q
+    if w.steps == 0:
+        return [(n_q, r, "none")]
     out = []
     for _ in range(w.steps):
+        kind = "fused"
         if r == R:
             n_q += R
             r = 0
+            kind = "flush"
         r += 1
-        out.append((n_q, r))
+        out.append((n_q, r, kind))
     return out
 
 
-def get_workload(args):
+def decode_schedule(w):
+    """(n_q, r) seen by each decode call of one layer's step, in order."""
+    return [(n_q, r) for n_q, r, _ in decode_calls(w)]
+
+
+def flush_steps(w):
+    """Per decode call, whether its append flushes the residual."""
+    return [kind == "flush" for _, _, kind in decode_calls(w)]
+
+
+def get_workload(args, name=None):
     from bit_asymmetric_kv_prefill_b200 import synth
-    w = synth.WORKLOADS[args.workload]
+    w = synth.WORKLOADS[name or args.workload]
     over = {}
-    if args.batch:
+    if name is None and args.batch:
         over["B"] = args.batch
-    if args.decode_steps:
+    if name is None and args.decode_steps:
         over["steps"] = args.decode_steps
     return synth.scaled(w, **over) if over else w
 
 
 def is_headline(args):
     return args.workload == WORKLOAD and not args.batch and not args.decode_steps
-
-
-def flush_steps(w):
-    """Per decode step, whether its append flushes the residual (n_q grows)."""
-    sched = decode_schedule(w)
-    n_q0 = w.R * ((w.T - 1) // w.R)
-    return [sched[j][0] != (sched[j - 1][0] if j else n_q0) for j in range(w.steps)]
 
 
 def decode_bytes(w, n_q, r):
@@ -101,8 +131,35 @@ def decode_bytes(w, n_q, r):
     return w.B * w.H_kv * (n_q * per_q + r * per_r) + w.B * w.H_q * w.D * (2 + 4)
 
 
+def fused_append_bytes(w):
+    """A fused launch also reads k_t, v_t and writes them to the residual."""
+    return 4 * w.B * w.H_kv * w.D * 2
+
+
+def prefill_bytes(w):
+    """Algorithmic HBM bytes of a prefill: K and V read once (2 B per element),
+    the packed groups written (24*D bytes per 32 quantized tokens of a
+    sequence: codes and fp16 scale/zero of keys and values) and the r residual
+    rows of K and V written."""
+    n_q = w.R * ((w.T - 1) // w.R)
+    r = w.T - n_q
+    seqs = w.B * w.H_kv
+    return seqs * (2 * w.T * w.D * 2 + (n_q // w.G) * 24 * w.D + 2 * r * w.D * 2)
+
+
 def decode_units(w, n_q, r):
     return w.B * w.H_kv * (n_q + r)
+
+
+def cache_record_bytes(w, layers):
+    """Per-token bytes of `layers` layer caches of capacity w.T, as the record
+    counts them: every context token's 2-bit codes plus a full R-slot residual
+    (and, separately, the fp16 scale/zero metadata)."""
+    per_layer_codes = w.B * w.H_kv * w.T * w.D * 2 * 2 // 8
+    per_layer_res = w.B * w.H_kv * w.R * w.D * 2 * 2
+    per_layer_meta = w.B * w.H_kv * w.T * 2 * (4 * w.D // w.G)
+    return (layers * (per_layer_codes + per_layer_res) / (w.B * w.T),
+            layers * per_layer_meta / (w.B * w.T))
 
 
 def source_hash():
@@ -130,13 +187,15 @@ def measured_peak():
         return 6650.0, "fallback"
 
 
-def traffic_per_launch(args):
-    """dram read+write bytes per decode launch from the committed ncu summary,
-    or None when absent, taken on other kernel sources or on another workload."""
-    if not is_headline(args):
+def traffic_per_launch(w, full_size):
+    """dram read+write bytes per decode launch from the committed ncu summary
+    of this workload, or None when absent, taken on other kernel sources or
+    when the workload was shrunk."""
+    path = PROFILE_TRAFFIC.get(w.name)
+    if not full_size or path is None:
         return None
     try:
-        with open(PROFILE_TRAFFIC) as f:
+        with open(path) as f:
             d = json.load(f)
     except Exception:
         return None
@@ -209,6 +268,12 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def clock_sampler(dev):
+    import torch
+    props = torch.cuda.get_device_properties(dev)
+    return ClockSampler(f"{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0")
+
+
 # ---- multi-rank helpers ------------------------------------------------------------
 
 def dist_env():
@@ -238,32 +303,79 @@ def barrier(device):
 
 # ---- CPU oracle leg ------------------------------------------------------------------
 
-def oracle_stream_rate(w, seconds: float, max_seqs: int = 1 << 30):
-    """Time the oracle on whole per-sequence streams (prefill + `steps` x
-    (append + decode)) of the workload until `seconds` elapse; returns
-    (units/s, sequences done, seconds)."""
-    import oracle
+def oracle_sample(w, steps=None):
+    """The oracle's unit of work: one (batch, kv head) sequence of the workload,
+    prefill of w.T tokens then its first `steps` decode calls (all by
+    default), each appending its token first.  Returns the one-sequence
+    workload, its calls and their KV token x head units."""
     from bit_asymmetric_kv_prefill_b200 import synth
-    sched = decode_schedule(w)
-    units_seq = sum(n_q + r for n_q, r in sched)
+    calls = decode_calls(w)
+    if steps is not None:
+        calls = calls[:max(1, steps)]
     one = synth.scaled(w, B=1, H_q=w.H_q // w.H_kv, H_kv=1)
-    done, t_used = 0, 0.0
+    return one, calls, sum(n_q + r for n_q, r, _ in calls)
+
+
+def _oracle_inputs(one, calls, seed):
+    from bit_asymmetric_kv_prefill_b200 import synth
+    K, V = synth.prefill_inputs(one, seed=seed)
+    steps = [tuple(synth.bits(x) for x in synth.step_inputs(one, s, seed=seed))
+             for s in range(1, len(calls) + 1)]
+    return synth.bits(K), synth.bits(V), steps
+
+
+def _oracle_sequence(one, w, calls, inp):
+    import oracle
+    kb, vb, steps = inp
     dt = oracle.DTYPE_BF16 if w.dtype == "bf16" else oracle.DTYPE_F16
-    while (t_used < seconds or done == 0) and done < max_seqs:
-        K, V = synth.prefill_inputs(one, seed=done)
-        kb, vb = synth.bits(K), synth.bits(V)
-        steps = [tuple(synth.bits(x) for x in synth.step_inputs(one, s, seed=done))
-                 for s in range(1, w.steps + 1)]
-        c = oracle.OracleCache(1, 1, w.D, w.G, w.R, dt, w.T_max, pre_rope=w.pre_rope,
-                               rope_theta=w.rope_theta)
-        t0 = time.perf_counter()
-        c.prefill(kb, vb)
-        for k, v, q in steps:
+    c = oracle.OracleCache(1, 1, w.D, w.G, w.R, dt, w.T_max, pre_rope=w.pre_rope,
+                           rope_theta=w.rope_theta)
+    c.prefill(kb, vb)
+    for (_, _, kind), (k, v, q) in zip(calls, steps):
+        if kind != "none":
             c.append(k, v)
-            c.decode(q)
-        t_used += time.perf_counter() - t0
-        done += 1
-    return units_seq * done / t_used, done, t_used
+        c.decode(q)
+
+
+def oracle_rate(w, seconds: float, threads: int, steps=None, waves: int = 0):
+    """Time the oracle on whole sequence samples (see oracle_sample) on
+    `threads` threads at once (each C call releases the GIL).  Threads loop
+    over samples until `seconds` have passed (at least one each), or run
+    exactly `waves` samples each.  Returns (units/s, samples done, wall s)."""
+    one, calls, units = oracle_sample(w, steps)
+    n_inputs = min(threads, 4)
+    inputs = [_oracle_inputs(one, calls, seed=i) for i in range(n_inputs)]
+    start = threading.Barrier(threads + 1)
+    done = [0] * threads
+    ends = [0.0] * threads
+    t0 = [0.0]
+
+    def worker(i):
+        start.wait()
+        n = 0
+        while True:
+            _oracle_sequence(one, w, calls, inputs[(i + n) % n_inputs])
+            n += 1
+            now = time.perf_counter()
+            if (waves and n >= waves) or (not waves and now - t0[0] >= seconds):
+                break
+        done[i] = n
+        ends[i] = now
+
+    ts = [threading.Thread(target=worker, args=(i,)) for i in range(threads)]
+    for t in ts:
+        t.start()
+    t0[0] = time.perf_counter()
+    start.wait()
+    for t in ts:
+        t.join()
+    wall = max(ends) - t0[0]
+    return units * sum(done) / wall, sum(done), wall
+
+
+def oracle_threads():
+    import oracle
+    return oracle.workers()
 
 
 def run_reference(args):
@@ -271,48 +383,229 @@ def run_reference(args):
     if rank != 0:
         return 0
     import oracle
-    from bit_asymmetric_kv_prefill_b200 import synth
     oracle.build()
     w = get_workload(args)
+    threads = oracle_threads()
+    k = ORACLE_STEPS.get(w.name)
+    _, calls, units = oracle_sample(w, k)
     for _ in range(args.warmup):
-        oracle_stream_rate(w, 0.0, max_seqs=1)
+        oracle_rate(w, 0.0, threads, k, waves=1)
     t_total, units_total = 0.0, 0.0
-    units_seq = sum(n_q + r for n_q, r in decode_schedule(w))
     for _ in range(args.steps):
-        _, n, t = oracle_stream_rate(w, 0.0, max_seqs=1)
+        _, n, t = oracle_rate(w, 0.0, threads, k, waves=1)
         t_total += t
-        units_total += units_seq * n
+        units_total += units * n
     value = units_total / t_total
-    sample = (f"each step: one (batch, head) sequence of {w.name}: prefill T={w.T} + "
-              f"{w.steps} x (append + decode), single thread")
+    sample = (f"each step: {threads} threads, each one (batch, kv head) sequence of {w.name}: "
+              f"prefill T={w.T} + {len(calls)} of its {len(decode_calls(w))} decode calls "
+              f"(append + decode)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_config(w, args),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "data": "synthetic", "config": workload_config(w, args, LAYERS[w.name], world),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
+def cpu_baseline(w, seconds):
+    """The oracle on the host's cores (and on one thread) over bounded samples
+    of the workload."""
+    threads = oracle_threads()
+    k = ORACLE_STEPS.get(w.name)
+    _, calls, _ = oracle_sample(w, k)
+    rate, n, wall = oracle_rate(w, seconds, threads, k)
+    rate1, n1, wall1 = oracle_rate(w, seconds / 3, 1, k)
+    what = (f"(batch, kv head) sequences of {w.name}, each prefill T={w.T} + the first "
+            f"{len(calls)} of its {len(decode_calls(w))} decode calls (append + decode)")
+    return {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{n} {what} on {threads} threads in {wall:.1f} s",
+            "single_thread": {"value": rate1, "unit": UNIT,
+                              "sample": f"{n1} such sequences on one thread in {wall1:.1f} s"}}
+
+
 # ---- GPU leg ----------------------------------------------------------------------------
 
-def workload_config(w, args):
+def workload_config(w, args, layers, world, sets=None):
     heads = f"{w.H_q} MHA heads" if w.H_q == w.H_kv else f"{w.H_q} query heads over {w.H_kv} kv heads"
-    title = "Llama-2-7B layer shape, " if w.name == WORKLOAD else ""
     rope = f", keys pre-RoPE (theta {w.rope_theta:g})" if w.pre_rope else ""
     per_layer = w.B * w.H_kv * (w.T_max * 2 * (w.D // 4 + 4 * w.D // w.G) + w.R * 4 * w.D)
-    ws_mb = args.layers * per_layer / 1e6
-    l2 = (f"inputs larger than L2: {args.layers} layer caches visited round-robin "
-          f"(~{ws_mb:.0f} MB working set vs 126 MB L2), no explicit flush") if ws_mb > 126 else \
-         f"working set {ws_mb:.0f} MB, not larger than L2 (126 MB)"
-    return {"workload": f"{w.name}: {title}batch {w.B}, {heads}, head_dim {w.D}, context {w.T}, "
-                        f"G={w.G}, R={w.R}, {w.dtype} input/residual{rope}, "
-                        f"prefill + {w.steps} x (append + decode) per layer",
-            "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "D": w.D, "T": w.T, "G": w.G, "R": w.R,
-            "decode_steps": w.steps, "layers_round_robin": args.layers, "l2": l2,
-            "parallelism": f"replicas x{max(1, args.gpus)} (no data-path collective)"}
+    ws_mb = layers * per_layer / 1e6
+    steps = (f"prefill + {w.steps} x (append + decode)" if w.steps else "prefill + one decode")
+    l2 = (f"inputs larger than L2: {layers} layer cache(s) of {per_layer / 1e6:.0f} MB visited "
+          f"round-robin (~{ws_mb:.0f} MB working set vs 126 MB L2), no explicit flush") \
+        if ws_mb > 126 else f"working set {ws_mb:.0f} MB, not larger than L2 (126 MB)"
+    cfg = {"workload": f"{w.name}: batch {w.B}, {heads}, head_dim {w.D}, context {w.T}, "
+                       f"G={w.G}, R={w.R}, {w.dtype} input/residual{rope}, {steps} per layer",
+           "B": w.B, "H_q": w.H_q, "H_kv": w.H_kv, "D": w.D, "T": w.T, "G": w.G, "R": w.R,
+           "decode_steps": w.steps, "layers_round_robin": layers, "l2": l2,
+           "parallelism": f"replicas x{max(1, world)} (no data-path collective)"}
+    if sets and sets < layers:
+        cfg["prefill_input_sets"] = sets
+    return cfg
+
+
+class Workbench:
+    """Caches and device-resident inputs of one workload, and its timed step."""
+
+    def __init__(self, w, layers, sets, rank, dev):
+        import torch
+        import bit_asymmetric_kv_prefill_b200 as kivi
+        from bit_asymmetric_kv_prefill_b200 import KiviCache, synth
+        self.w, self.nl, self.dev = w, layers, dev
+        self.sets = min(sets, layers)
+        self.L = kivi.lib()
+        self.calls = decode_calls(w)
+        self.caches = [KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, w.T_max,
+                                 pre_rope=w.pre_rope, rope_theta=w.rope_theta)
+                       for _ in range(layers)]
+        self.Ks, self.Vs = [], []
+        for l in range(self.sets):
+            K, V = synth.prefill_inputs(w, seed=1000 * rank + l, device=dev)
+            self.Ks.append(K)
+            self.Vs.append(V)
+        # per call, per input set: (k_t, v_t, q)
+        self.steps = [[synth.step_inputs(w, max(s, 1), seed=1000 * rank + l, device=dev)
+                       for l in range(self.sets)] for s in range(1, len(self.calls) + 1)]
+        self.outs = [torch.empty(w.B, w.H_q, w.D, dtype=torch.float32, device=dev)
+                     for _ in range(layers)]
+        self.stream = torch.cuda.current_stream(dev)
+        self.sp = ctypes.c_void_p(self.stream.cuda_stream)
+        self.H = [c._h for c in self.caches]
+        self.Kp = [ctypes.c_void_p(t.data_ptr()) for t in self.Ks]
+        self.Vp = [ctypes.c_void_p(t.data_ptr()) for t in self.Vs]
+        self.Sp = [[tuple(ctypes.c_void_p(t.data_ptr()) for t in st) for st in row]
+                   for row in self.steps]
+        self.Op = [ctypes.c_void_p(o.data_ptr()) for o in self.outs]
+        self.units_step = sum(decode_units(w, n, r) for n, r, _ in self.calls) * layers
+        self.bytes_step = (sum(decode_bytes(w, n, r) for n, r, _ in self.calls)
+                           + fused_append_bytes(w) * sum(k == "fused" for _, _, k in self.calls)) * layers
+        self.n_dec = layers * len(self.calls)
+        self.launches_step = layers * (1 + len(self.calls) + sum(k == "flush" for _, _, k in self.calls))
+
+    def step(self, dec_ev=None, pre_ev=None):
+        """One step: every layer's reset and prefill, then the decode calls.
+        Events (CUDA, on the launching stream) bracket each decode launch and
+        each prefill when given."""
+        L, H, sp, w = self.L, self.H, self.sp, self.w
+        bad = 0
+        for l in range(self.nl):
+            i = l % self.sets
+            bad |= L.kivi_cache_reset(H[l])
+            if pre_ev is not None:
+                pre_ev[l][0].record(self.stream)
+            bad |= L.kivi_prefill(H[l], self.Kp[i], self.Vp[i], w.T, sp)
+            if pre_ev is not None:
+                pre_ev[l][1].record(self.stream)
+        j = 0
+        for c, (_, _, kind) in enumerate(self.calls):
+            row = self.Sp[c]
+            for l in range(self.nl):
+                k, v, q = row[l % self.sets]
+                if kind == "flush":
+                    bad |= L.kivi_append(H[l], k, v, sp)
+                if dec_ev is not None:
+                    dec_ev[j][0].record(self.stream)
+                if kind == "fused":
+                    bad |= L.kivi_append_decode(H[l], k, v, q, w.H_q, self.Op[l], sp)
+                else:
+                    bad |= L.kivi_decode_attn(H[l], q, w.H_q, self.Op[l], sp)
+                if dec_ev is not None:
+                    dec_ev[j][1].record(self.stream)
+                j += 1
+        if bad:
+            raise RuntimeError("a KIVI call failed during the benchmark")
+
+    def measure(self, steps, warmup, clocks=True):
+        """Warm up, then time `steps` steps (device time of the whole region,
+        and of every decode launch and prefill).  Returns a dict of timings."""
+        import torch
+        for _ in range(warmup):
+            self.step()
+        ev = lambda: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+        dec_ev = [[ev() for _ in range(self.n_dec)] for _ in range(steps)]
+        pre_ev = [[ev() for _ in range(self.nl)] for _ in range(steps)]
+        t0e, t1e = ev()
+        ck = clock_sampler(self.dev) if clocks else None
+        barrier(self.dev)
+        if ck:
+            ck.start()
+            time.sleep(0.3)  # let the sampler attach before the timed region
+        t0e.record(self.stream)
+        for k in range(steps):
+            self.step(dec_ev[k], pre_ev[k])
+        t1e.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        cks = ck.stop() if ck else None
+        barrier(self.dev)
+        status = max(c.device_status() for c in self.caches)
+        if status != 0:
+            raise RuntimeError(f"device status {status} after the timed region")
+        dec_ms = [a.elapsed_time(b) for row in dec_ev for a, b in row]
+        pre_ms = [a.elapsed_time(b) for row in pre_ev for a, b in row]
+        return {"ms": t0e.elapsed_time(t1e), "dec_ms": dec_ms, "pre_ms": pre_ms, "clocks": cks}
+
+    def close(self):
+        for c in self.caches:
+            c.close()
+
+
+def summarize(wb, t, steps, world, peak):
+    """Per-workload figures from a Workbench measurement."""
+    w = wb.w
+    dec_avg = sum(t["dec_ms"]) / len(t["dec_ms"])
+    pre_avg = sum(t["pre_ms"]) / len(t["pre_ms"])
+    bpl = wb.bytes_step / wb.n_dec
+    achieved = bpl / (dec_avg / 1e3) / 1e9
+    pb = prefill_bytes(w)
+    return {
+        "value": world * wb.units_step * steps / (t["ms"] / 1e3), "unit": UNIT,
+        "ms_per_step": t["ms"] / steps, "steps": steps,
+        "decode": {"avg_us": 1e3 * dec_avg, "median_us": 1e3 * statistics.median(t["dec_ms"]),
+                   "p90_us": 1e3 * sorted(t["dec_ms"])[int(0.9 * (len(t["dec_ms"]) - 1))],
+                   "launches_timed": len(t["dec_ms"]), "alg_bytes_per_launch": bpl,
+                   "achieved_gbs": achieved, "frac_of_measured_hbm": achieved / peak,
+                   "frac_of_8TBps": achieved / 8000.0,
+                   "tokens_heads_per_s": wb.units_step / wb.n_dec / (dec_avg / 1e3),
+                   "gpu_time_share": sum(t["dec_ms"]) / t["ms"]},
+        "prefill": {"avg_us": 1e3 * pre_avg, "alg_bytes": pb,
+                    "achieved_gbs": pb / (pre_avg / 1e3) / 1e9,
+                    "frac_of_measured_hbm": pb / (pre_avg / 1e3) / 1e9 / peak,
+                    "launches_timed": len(t["pre_ms"])},
+        "clocks": t["clocks"],
+    }
+
+
+def per_config_entry(args, name, dev, peak):
+    """Measure one of the other workloads at full size (rank 0, N = 1)."""
+    import torch
+    w = get_workload(args, name)
+    layers, sets = LAYERS[name], INPUT_SETS.get(name, LAYERS[name])
+    wb = Workbench(w, layers, sets, 0, dev)
+    try:
+        t = wb.measure(args.steps, args.warmup)
+        s = summarize(wb, t, args.steps, 1, peak)
+        s["config"] = workload_config(w, args, layers, 1, sets)
+        s["gpu_launches"] = wb.launches_step * args.steps
+        tr = traffic_per_launch(w, True)
+        s["decode"]["traffic"] = tr
+        if name == "llama2_13b_cache":
+            nb = wb.caches[0].nbytes()
+            per_tok = lambda x: x * layers / (w.B * w.T)
+            rec, meta = cache_record_bytes(w, layers)
+            s["cache_bytes"] = {
+                "codes_plus_residual_per_token": per_tok(nb["codes"] + nb["residual"]),
+                "metadata_per_token": per_tok(nb["meta"]),
+                "record_per_token": 128000, "record_basis_closed_form": rec,
+                "matches_record": per_tok(nb["codes"] + nb["residual"]) == 128000 == rec,
+                "source": "kivi_cache_bytes of the allocated caches (capacity 4,096 tokens)"}
+        return s
+    finally:
+        wb.close()
+        del wb
+        torch.cuda.empty_cache()
 
 
 def run_gpu(args):
@@ -326,152 +619,68 @@ def run_gpu(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    import bit_asymmetric_kv_prefill_b200 as kivi
-    from bit_asymmetric_kv_prefill_b200 import KiviCache, synth
     from bit_asymmetric_kv_prefill_b200 import build as kbuild
     kbuild.build()
-    L = kivi.lib()
 
     w = get_workload(args)
-    nl = args.layers
-    sched = decode_schedule(w)
-    # A fused launch also reads k_t, v_t and writes them to the residual.
-    fused_extra = 4 * w.B * w.H_kv * w.D * 2 * (w.steps - sum(flush_steps(w)))
-    bytes_step = (sum(decode_bytes(w, n, r) for n, r in sched) + fused_extra) * nl
-    units_step = sum(decode_units(w, n, r) for n, r in sched) * nl
-    launches_step = nl * (1 + w.steps + sum(flush_steps(w)))
-
-    caches = [KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, w.T_max, pre_rope=w.pre_rope,
-                        rope_theta=w.rope_theta) for _ in range(nl)]
-    Ks, Vs = [], []
-    for l in range(nl):
-        K, V = synth.prefill_inputs(w, seed=1000 * rank + l, device=dev)
-        Ks.append(K)
-        Vs.append(V)
-    steps = [[synth.step_inputs(w, s, seed=1000 * rank + l, device=dev) for l in range(nl)]
-             for s in range(1, w.steps + 1)]
-    outs = [torch.empty(w.B, w.H_q, w.D, dtype=torch.float32, device=dev) for _ in range(nl)]
-    stream = torch.cuda.current_stream(dev)
-    sp = ctypes.c_void_p(stream.cuda_stream)
-    H = [c._h for c in caches]
-    Kp = [ctypes.c_void_p(t.data_ptr()) for t in Ks]
-    Vp = [ctypes.c_void_p(t.data_ptr()) for t in Vs]
-    Sp = [[tuple(ctypes.c_void_p(t.data_ptr()) for t in st) for st in row] for row in steps]
-    Op = [ctypes.c_void_p(o.data_ptr()) for o in outs]
-    T, Hq = w.T, w.H_q
-    reset, prefill, append, decode, fused = (L.kivi_cache_reset, L.kivi_prefill, L.kivi_append,
-                                             L.kivi_decode_attn, L.kivi_append_decode)
-    # Steps whose append flushes (the quantizer runs): append, then decode;
-    # the others fuse the append into the decode launch.  Either way the timed
-    # launch is one decode.
-    flush = flush_steps(w)
-
-    def one_step(ev=None):
-        bad = 0
-        for l in range(nl):
-            bad |= reset(H[l])
-            bad |= prefill(H[l], Kp[l], Vp[l], T, sp)
-        i = 0
-        for j, row in enumerate(Sp):
-            for l in range(nl):
-                k, v, q = row[l]
-                if flush[j]:
-                    bad |= append(H[l], k, v, sp)
-                if ev is not None:
-                    ev[i][0].record(stream)
-                if flush[j]:
-                    bad |= decode(H[l], q, Hq, Op[l], sp)
-                else:
-                    bad |= fused(H[l], k, v, q, Hq, Op[l], sp)
-                if ev is not None:
-                    ev[i][1].record(stream)
-                i += 1
-        if bad:
-            raise RuntimeError("a KIVI call failed during the benchmark")
-
-    for _ in range(args.warmup):
-        one_step()
-    n_dec = nl * w.steps
-    events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-               for _ in range(n_dec)] for _ in range(args.steps)]
-    t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    props = torch.cuda.get_device_properties(dev)
-    clocks = ClockSampler(f"{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0")
-    barrier(dev)
-    clocks.start()
-    time.sleep(0.3)  # let the sampler attach before the timed region
-    t0e.record(stream)
-    for k in range(args.steps):
-        one_step(events[k])
-    t1e.record(stream)
-    torch.cuda.synchronize(dev)
-    ck = clocks.stop()
-    barrier(dev)
-    ms_local = t0e.elapsed_time(t1e)
-    dec_ms = [a.elapsed_time(b) for ev in events for a, b in ev]
-    dec_avg_local = sum(dec_ms) / len(dec_ms)
-    status = max(c.device_status() for c in caches)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed region")
-
-    ms = reduce_max(ms_local, dev)
-    dec_avg = reduce_max(dec_avg_local, dev)
-    value = world * units_step * args.steps / (ms / 1e3)
-    bytes_per_launch = bytes_step / n_dec
-    achieved = bytes_per_launch / (dec_avg / 1e3) / 1e9
+    layers = args.layers or LAYERS[w.name]
+    sets = min(INPUT_SETS.get(w.name, layers), layers)
     peak, peak_kind = measured_peak()
-    traffic = traffic_per_launch(args)
+    wb = Workbench(w, layers, sets, rank, dev)
+    t = wb.measure(args.steps, args.warmup)
+    ms = reduce_max(t["ms"], dev)
+    dec_avg = reduce_max(sum(t["dec_ms"]) / len(t["dec_ms"]), dev)
+    t["ms"] = ms
+    s = summarize(wb, t, args.steps, world, peak)
+    achieved = s["decode"]["alg_bytes_per_launch"] / (dec_avg / 1e3) / 1e9
+    e2e = run_e2e(args, wb, world) if sets == layers else None
+    launches = wb.launches_step * args.steps
+    wb.close()
+    del wb
+    torch.cuda.empty_cache()
 
-    e2e = run_e2e(args, w, caches, Ks, Vs, steps, dev, world)
-
-    cpu = None
+    per_config, cpu = None, None
+    if world == 1 and is_headline(args) and not args.no_per_config:
+        per_config = {name: per_config_entry(args, name, dev, peak) for name in PER_CONFIG}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, nseq, secs = oracle_stream_rate(w, args.cpu_seconds)
-        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{nseq} (batch, head) sequences of {w.name}, each prefill T={w.T} + "
-                         f"{w.steps} x (append + decode); {secs:.1f} s single-threaded"}
+        cpu = cpu_baseline(w, args.cpu_seconds)
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "metric": METRIC, "value": s["value"], "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
-            "data": "synthetic", "config": workload_config(w, args),
+            "data": "synthetic", "config": workload_config(w, args, layers, world, sets),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic,
+                         "frac": achieved / peak,
+                         "traffic": traffic_per_launch(w, not (args.batch or args.decode_steps)),
                          "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                         "kernel": "decode_kernel (kivi_decode_attn)",
-                         "alg_bytes_per_launch": bytes_per_launch,
+                         "kernel": "decode_kernel (kivi_decode_attn / kivi_append_decode)",
+                         "alg_bytes_per_launch": s["decode"]["alg_bytes_per_launch"],
                          "frac_of_8TBps": achieved / 8000.0},
-            "decode_attn": {"avg_us": 1e3 * dec_avg,
-                            "median_us": 1e3 * statistics.median(dec_ms),
-                            "p90_us": 1e3 * sorted(dec_ms)[int(0.9 * (len(dec_ms) - 1))],
-                            "launches_timed": len(dec_ms),
-                            "tokens_heads_per_s": units_step / nl / w.steps / (dec_avg / 1e3),
-                            "gpu_time_share": sum(dec_ms) / ms_local},
-            "e2e": e2e, "gpu_launches": launches_step * args.steps, "clocks": ck,
-            "cpu_baseline": cpu,
+            "decode_attn": s["decode"], "prefill": s["prefill"],
+            "e2e": e2e, "gpu_launches": launches, "clocks": s["clocks"],
+            "cpu_baseline": cpu, "per_config": per_config,
         }
         print(json.dumps(line), flush=True)
-    for c in caches:
-        c.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
 
 
-def run_e2e(args, w, caches, Ks, Vs, steps, dev, world):
+def run_e2e(args, wb, world):
     """Same step through the public API with pinned HOST inputs: the H2D copies
     of every input and the D2H read of every decode output are timed.
 
-    Copies run on their own stream, as a serving loop would run them: step
+    Copies run on their own streams, as a serving loop would run them: step
     k+1's prefill inputs stream in while step k computes (each layer's buffer
     is refilled once that layer's prefill has read it), and each step's decode
     inputs land in one of two buffer sets.  Every timed step's copies happen
     inside the timed region; outputs return on the compute stream."""
     import torch
-    nl = len(caches)
+    w, dev, nl, caches = wb.w, wb.dev, wb.nl, wb.caches
+    Ks, Vs, steps = wb.Ks, wb.Vs, [[row[l] for l in range(nl)] for row in wb.steps]
     hK = [k.cpu().pin_memory() for k in Ks]
     hV = [v.cpu().pin_memory() for v in Vs]
     hS = [[tuple(t.cpu().pin_memory() for t in st) for st in row] for row in steps]
@@ -490,6 +699,7 @@ def run_e2e(args, w, caches, Ks, Vs, steps, dev, world):
     ev_sused = [torch.cuda.Event() for _ in range(2)]
     for e in ev_used + ev_sused:
         e.record(cs)
+    kinds = [kind for _, _, kind in wb.calls]
 
     def copies(k):
         b = k % 2
@@ -522,7 +732,10 @@ def run_e2e(args, w, caches, Ks, Vs, steps, dev, world):
         for j in range(len(hS)):
             for l in range(nl):
                 k_t, v_t, q = dS[b][j][l]
-                out = caches[l].append_decode(k_t, v_t, q)
+                if kinds[j] == "none":
+                    out = caches[l].decode(q)
+                else:
+                    out = caches[l].append_decode(k_t, v_t, q)
                 hout[l].copy_(out, non_blocking=True)
         ev_sused[b].record(cs)
 
@@ -544,10 +757,9 @@ def run_e2e(args, w, caches, Ks, Vs, steps, dev, world):
     torch.cuda.synchronize(dev)
     barrier(dev)
     ms = reduce_max(a.elapsed_time(b), dev)
-    sched = decode_schedule(w)
-    units = sum(decode_units(w, nq, r) for nq, r in sched) * nl
-    h2d = nl * (2 * Ks[0].numel() * 2 + w.steps * sum(t.numel() * 2 for t in steps[0][0]))
-    d2h = nl * w.steps * w.B * w.H_q * w.D * 4
+    units = wb.units_step
+    h2d = nl * (2 * Ks[0].numel() * 2 + len(hS) * sum(t.numel() * 2 for t in steps[0][0]))
+    d2h = nl * len(hS) * w.B * w.H_q * w.D * 4
     return {"value": world * units * n / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": ms / n,
             "copies": "H2D on two copy streams (keys, values), step k+1's inputs during step k"}
@@ -679,15 +891,17 @@ def run_diag(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kivi", "reference"], default="kivi")
-    ap.add_argument("--layers", type=int, default=8)
-    ap.add_argument("--e2e-steps", dest="e2e_steps", type=int, default=5)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layer caches per step (default: the workload's own count)")
+    ap.add_argument("--e2e-steps", dest="e2e_steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", dest="cpu_seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", dest="no_cpu_baseline", action="store_true")
-    ap.add_argument("--workload", default=WORKLOAD,
-                    choices=["tiny", "llama2_7b_layer", "llama2_13b_cache", "mistral_gqa", "long_context"])
+    ap.add_argument("--no-per-config", dest="no_per_config", action="store_true",
+                    help="skip the other workloads' measurements")
+    ap.add_argument("--workload", default=WORKLOAD, choices=WORKLOAD_NAMES)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
     ap.add_argument("--decode-steps", dest="decode_steps", type=int, default=0,
                     help="override the workload's decode steps")

@@ -17,6 +17,7 @@ from __future__ import annotations
 import ctypes
 import os
 import subprocess
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -78,6 +79,39 @@ def lib():
     L.oracle_float_to_f16.restype = ctypes.c_uint16
     _lib = L
     return L
+
+
+def workers() -> int:
+    """Threads the oracle runs sequences on: the CPUs this process may use
+    (``KIVI_ORACLE_THREADS`` overrides).  Each (batch, kv head) sequence is
+    one C call, and ctypes releases the GIL for the call's duration, so the
+    sequences of a cache run in parallel; none shares memory with another,
+    and every result is the same as with one thread."""
+    env = os.environ.get("KIVI_ORACLE_THREADS")
+    if env:
+        return max(1, int(env))
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+_pool = None
+
+
+def parallel_map(fn, items, threads=None):
+    """list(map(fn, items)) on up to `threads` (default workers()) threads."""
+    items = list(items)
+    n = workers() if threads is None else threads
+    if n <= 1 or len(items) <= 1:
+        return [fn(x) for x in items]
+    global _pool
+    if threads is not None:
+        with ThreadPoolExecutor(n) as ex:
+            return list(ex.map(fn, items))
+    if _pool is None:
+        _pool = ThreadPoolExecutor(n)
+    return list(_pool.map(fn, items))
 
 
 def _ptr(a: np.ndarray, ct):
@@ -258,15 +292,19 @@ class OracleCache:
         if len(lengths) != self.B or min(lengths) < 1 or max(lengths) > T:
             raise ValueError(f"lengths must be {self.B} values in [1, {T}], got {lengths}")
         L = lib()
-        nq, r = ctypes.c_longlong(), ctypes.c_int()
-        for b in range(self.B):
-            for h in range(self.H):
-                kb = np.ascontiguousarray(K[b, h, :lengths[b]])
-                vb = np.ascontiguousarray(V[b, h, :lengths[b]])
-                L.oracle_prefill_seq(_ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
-                                     lengths[b], self.D, self.G, self.R, self.dtype,
-                                     *self._seq_ptrs(b, h), ctypes.byref(nq), ctypes.byref(r))
-            self.nqb[b], self.rb[b] = nq.value, r.value
+
+        def one(bh):
+            b, h = bh
+            nq, r = ctypes.c_longlong(), ctypes.c_int()
+            kb = np.ascontiguousarray(K[b, h, :lengths[b]])
+            vb = np.ascontiguousarray(V[b, h, :lengths[b]])
+            L.oracle_prefill_seq(_ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+                                 lengths[b], self.D, self.G, self.R, self.dtype,
+                                 *self._seq_ptrs(b, h), ctypes.byref(nq), ctypes.byref(r))
+            return b, nq.value, r.value
+
+        for b, nq, r in parallel_map(one, [(b, h) for b in range(self.B) for h in range(self.H)]):
+            self.nqb[b], self.rb[b] = nq, r
 
     def append(self, k: np.ndarray, v: np.ndarray):
         """k, v: uint16 bit patterns [B, H_kv, D]."""
@@ -292,10 +330,12 @@ class OracleCache:
         B, H_q, D = q.shape
         HG = H_q // self.H
         out = np.full((B, H_q, D), np.nan, np.float32)
-        sc = np.zeros(max(int((self.nqb + self.rb).max()), 1), np.float64)
         L = lib()
         pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(self.H)]
-        for b, h in pairs:
+
+        def one(bh):
+            b, h = bh
+            sc = np.zeros(max(int(self.nqb[b] + self.rb[b]), 1), np.float64)
             qb = np.ascontiguousarray(q[b, h * HG:(h + 1) * HG])
             ob = np.zeros((HG, D), np.float32)
             L.oracle_decode_seq(_ptr(qb, ctypes.c_uint16), HG, D, self.G, self.R, self.dtype,
@@ -303,6 +343,8 @@ class OracleCache:
                                 int(self.nqb[b]), int(self.rb[b]), _ptr(sc, ctypes.c_double),
                                 _ptr(ob, ctypes.c_float))
             out[b, h * HG:(h + 1) * HG] = ob
+
+        parallel_map(one, pairs)
         return out
 
     def quantized(self):

@@ -8,3 +8,11 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_report_header(config):
+    try:
+        import oracle
+        return f"oracle threads: {oracle.workers()}"
+    except Exception as e:  # the header is informational only
+        return f"oracle threads: unknown ({e})"

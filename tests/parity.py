@@ -36,22 +36,49 @@ def assert_attn_close(out, ref, what=""):
     return rel, mabs
 
 
-def assert_store_equal(cache: KiviCache, orc: oracle.OracleCache, seqs):
+def _runs(seqs, chunk):
+    """Consecutive runs (first, count) of the sorted sequence list, at most
+    `chunk` long."""
+    seqs = sorted(seqs)
+    runs, i = [], 0
+    while i < len(seqs):
+        j = i
+        while j + 1 < len(seqs) and seqs[j + 1] == seqs[j] + 1 and j + 1 - i < chunk:
+            j += 1
+        runs.append((seqs[i], j - i + 1))
+        i = j + 1
+    return runs
+
+
+def assert_store_equal(cache: KiviCache, orc: oracle.OracleCache, seqs, chunk=8, orc_index=None):
     """Bit-exact comparison of the quantized store and residual of the given
-    flattened sequences (b*H_kv + h) of the GPU cache with an oracle cache that
-    holds every sequence."""
+    flattened sequences (b*H_kv + h) of the GPU cache with an oracle cache.
+    The oracle holds every sequence, or (orc_index) maps GPU sequence s to the
+    oracle's sequence orc_index[s].  The GPU store is exported in runs of
+    `chunk` sequences on the oracle's threads (the export is a C call that
+    releases the GIL)."""
     assert cache.length() == (orc.n_q, orc.r)
     ref = orc.quantized()
-    for s in seqs:
-        got = cache.export(s, 1)
-        ob, oh = divmod(s, orc.H)
-        for key in ("codesK", "codesV", "sK", "zK", "sV", "zV", "resK", "resV"):
-            a, b = got[key][0], ref[key][ob, oh]
-            if not np.array_equal(a, b):
-                bad = np.argwhere(a != b)
-                raise AssertionError(f"{key} differs for sequence {s} at {bad[:5].tolist()} "
-                                     f"({len(bad)} entries): gpu {a[tuple(bad[0])]} "
-                                     f"oracle {b[tuple(bad[0])]}")
+    keys = ("codesK", "codesV", "sK", "zK", "sV", "zV", "resK", "resV")
+
+    def one(run):
+        s0, n = run
+        got = cache.export(s0, n)
+        for i in range(n):
+            s = s0 + i
+            o = s if orc_index is None else orc_index[s]
+            ob, oh = divmod(o, orc.H)
+            for key in keys:
+                a, b = got[key][i], ref[key][ob, oh]
+                if not np.array_equal(a, b):
+                    bad = np.argwhere(a != b)
+                    return (f"{key} differs for sequence {s} at {bad[:5].tolist()} "
+                            f"({len(bad)} entries): gpu {a[tuple(bad[0])]} oracle {b[tuple(bad[0])]}")
+        return None
+
+    errs = [e for e in oracle.parallel_map(one, _runs(seqs, chunk)) if e]
+    if errs:
+        raise AssertionError(errs[0] + (f" (and {len(errs) - 1} more runs)" if len(errs) > 1 else ""))
 
 
 class Pair:
@@ -94,12 +121,20 @@ class Pair:
         self.cache.append(k, v)
         self.orc.append(self._pick(k), self._pick(v))
 
-    def decode(self, q):
-        """GPU output restricted to the oracle's sequences, and the oracle's."""
+    def decode(self, q, seqs=None):
+        """GPU output restricted to the oracle's sequences, and the oracle's;
+        `seqs` (flattened b*H_kv + h, oracle holding every sequence) restricts
+        both to those sequences' query heads."""
         out = self.cache.decode(q)
         torch.cuda.synchronize()
-        ref = self.orc.decode(self._pick_q(q))
         o = out.cpu().numpy()
+        if seqs is not None:
+            assert self.sample is None
+            H, HG = self.w.H_kv, self.HG
+            ref = self.orc.decode(synth.bits(q), heads=[divmod(s, H) for s in seqs])
+            rows = lambda a: np.stack([a[s // H, (s % H) * HG:(s % H + 1) * HG] for s in seqs])
+            return rows(o), rows(ref)
+        ref = self.orc.decode(self._pick_q(q))
         if self.sample is None:
             return o, ref
         HG = self.HG
@@ -113,13 +148,8 @@ class Pair:
             assert_store_equal(self.cache, self.orc, seqs)
         else:
             # oracle sequence i <-> GPU sequence sample[i]
-            assert self.cache.length() == (self.orc.n_q, self.orc.r)
-            ref = self.orc.quantized()
-            for i, s in enumerate(self.sample):
-                got = self.cache.export(s, 1)
-                for key in ref:
-                    if not np.array_equal(got[key][0], ref[key][i, 0]):
-                        raise AssertionError(f"{key} differs for sequence {s}")
+            assert_store_equal(self.cache, self.orc, seqs,
+                               orc_index={s: i for i, s in enumerate(self.sample)})
 
 
 def _vals(bits, dtype):

@@ -71,3 +71,37 @@ def test_decode_bytes_long_context():
 def test_units_are_kv_tokens_times_heads():
     w = W["llama2_7b_layer"]
     assert bench.decode_units(w, 4096, 5) == 8 * 32 * 4101
+
+
+def test_workloads_without_decode_steps_decode_once_over_the_prefill():
+    w = W["llama2_13b_cache"]
+    assert bench.decode_calls(w) == [(3968, 128, "none")]
+    assert bench.flush_steps(w) == [False]
+
+
+def test_decode_calls_mark_flushes_and_fused_appends():
+    kinds = [k for _, _, k in bench.decode_calls(W["mistral_gqa"])]
+    assert kinds.count("flush") == 2 and kinds[0] == kinds[128] == "flush"
+    assert kinds.count("fused") == 254
+
+
+def test_prefill_bytes_of_the_128k_pre_rope_context():
+    # 8 kv heads x 131,072 tokens x 128 channels of K and V read (bf16), 4,092
+    # packed groups of 3,072 B and 128 residual rows of K and V per sequence
+    w = W["long_context"]
+    assert bench.prefill_bytes(w) == 637_960_192
+    assert bench.prefill_bytes(w) == 8 * (2 * 131072 * 128 * 2 + 4092 * 3072 + 2 * 128 * 128 * 2)
+
+
+def test_cache_record_bytes_of_the_llama2_13b_cache():
+    # record kv-efficiency/kivi-2bit-llama2-13b-mha-4k, "KV bytes basis": 40
+    # layers at 4,096 tokens hold 128,000 B/token of codes and residual; fp16
+    # scale/zero per 32 add 51,200 B/token
+    assert bench.cache_record_bytes(W["llama2_13b_cache"], 40) == (128_000, 51_200)
+
+
+def test_oracle_sample_units():
+    w = W["mistral_gqa"]
+    one, calls, units = bench.oracle_sample(w, 8)
+    assert (one.B, one.H_kv, one.H_q) == (1, 1, 4) and len(calls) == 8
+    assert units == sum(n + r for n, r, _ in bench.decode_calls(w)[:8])
