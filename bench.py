@@ -70,6 +70,7 @@ PROFILE_TRAFFIC = {
     "mistral_gqa": os.path.join(ROOT, "profiles", "decode_mistral_gqa_traffic.json"),
 }
 DECODE_SOURCES = ["bit_asymmetric_kv_prefill_b200/csrc/kivi_decode.cu",
+                  "bit_asymmetric_kv_prefill_b200/csrc/kivi_decode_ops.cuh",
                   "bit_asymmetric_kv_prefill_b200/csrc/kivi_common.cuh"]
 
 

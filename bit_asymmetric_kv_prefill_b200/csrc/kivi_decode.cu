@@ -39,6 +39,7 @@
 #include <cuda_runtime.h>
 
 #include "kivi_common.cuh"
+#include "kivi_decode_ops.cuh"
 #include "kivi_internal.h"
 
 namespace kivi {
@@ -56,14 +57,13 @@ namespace kivi {
 #ifndef KIVI_DECODE_MAXW_GQA_ROPE
 #define KIVI_DECODE_MAXW_GQA_ROPE 8   // the same with pre-RoPE keys
 #endif
+#ifndef KIVI_KEYS_SCALAR
+#define KIVI_KEYS_SCALAR 1   // four query heads: key dot products as scalar FMAs
+#endif
 #ifndef KIVI_ROPE_UNROLL
 #define KIVI_ROPE_UNROLL 1   // pre-RoPE key loop: pair-steps unrolled (measured best)
 #endif
-#ifndef KIVI_SCALAR_F32
-#define KIVI_SCALAR_F32 0
-#endif
 
-constexpr unsigned FULL = 0xffffffffu;
 constexpr int kRopeUnroll = KIVI_ROPE_UNROLL;
 #ifndef KIVI_DECODE_STAGES_GQA
 #define KIVI_DECODE_STAGES_GQA 3   // four or more query heads per kv head
@@ -77,232 +77,6 @@ constexpr int ring_stages()
 {
     return HG >= 4 ? (ROPE ? KIVI_DECODE_STAGES_GQA_ROPE : KIVI_DECODE_STAGES_GQA) : KIVI_DECODE_STAGES;
 }
-constexpr float kRescaleSlack = 8.0f;
-constexpr int kWaitLimit = 1 << 22;
-
-// ---- PTX wrappers ----------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_addr(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, int count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
-                                         uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst),
-        "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-// Lane 0 of the calling warp arms `bar` for `bytes` and starts one bulk copy
-// of `bytes` into it; the other lanes skip both under a predicate (no branch).
-__device__ __forceinline__ void lane0_expect_copy(int lane, uint32_t bar, uint32_t dst, const void *src,
-                                                  uint32_t bytes, uint32_t expect)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, %0, 0;\n\t"
-        "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%1], %5;\n\t"
-        "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%2], [%3], %4, [%1];\n\t}"
-        ::"r"(lane), "r"(bar), "r"(dst), "l"(src), "r"(bytes), "r"(expect)
-        : "memory");
-}
-__device__ __forceinline__ void lane0_copy(int lane, uint32_t bar, uint32_t dst, const void *src,
-                                           uint32_t bytes)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, %0, 0;\n\t"
-        "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%2], [%3], %4, [%1];\n\t}"
-        ::"r"(lane), "r"(bar), "r"(dst), "l"(src), "r"(bytes)
-        : "memory");
-}
-__device__ __forceinline__ float ex2(float x)
-{
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
-{
-#if KIVI_SCALAR_F32
-    return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
-#endif
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-    return d;
-}
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
-{
-#if KIVI_SCALAR_F32
-    return make_float2(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y));
-#endif
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-
-// ---- code extraction ---------------------------------------------------------
-// Code pair i of a word (split-pair layout): first code at bits 2i of w,
-// second at bits 2i of w16 = w >> 16.  OR-ing the field into the mantissa of
-// 2^23 (`magic`, a runtime register so that the mask stays an immediate) gives
-// 2^23 + c*2^(2i) exactly; adding `neg` = (-2^23, -2^23) leaves
-// (c_first 2^(2i), c_second 2^(2i)).  One logic op per code; the power of two
-// is folded into the scales (the pre-RoPE key path uses this conversion,
-// since it dequantizes explicitly).
-__device__ __forceinline__ float2 code_pair(uint32_t w, uint32_t w16, int i, uint32_t magic,
-                                            float2 neg)
-{
-    const uint32_t msk = 3u << (2 * i);
-    uint32_t a, b;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(a) : "r"(w), "r"(msk), "r"(magic));
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(b) : "r"(w16), "r"(msk), "r"(magic));
-    return fadd2(make_float2(__uint_as_float(a), __uint_as_float(b)), neg);
-}
-// 2^-2i, the inverse of pair i's shift.
-__device__ __forceinline__ float pair_scale(int i) { return __uint_as_float((uint32_t)(127 - 2 * i) << 23); }
-// 2^e for -126 <= e <= 127.
-__device__ __forceinline__ float pow2i(int e) { return __uint_as_float((uint32_t)(127 + e) << 23); }
-
-// Keys, fast path: AND-ing pair i's field out of the word (or of the word
-// shifted right by 16) leaves the fp32 denormal c * 2^(2i-149).  Multiplying
-// by q'' = q' * 2^(kKexp-2i) gives q' c 2^(kKexp-149) with no conversion
-// step; one logic op per code and one fp32x2 FMA per pair.
-constexpr int kKexp = 64;
-constexpr float kKunscale = 0x1p85f;   // 2^(149 - kKexp)
-__device__ __forceinline__ float kq_scale(int i) { return pow2i(kKexp - 2 * i); }
-
-// Values: AND-ing 0x00030003 << 2j out of a word leaves two f16 subnormals
-// c * 2^(2j-24) in its halves (j <= 3; pairs 4..7 are read from the word
-// shifted right by 8).  They multiply an f16 token weight in a mixed-precision
-// FMA (exact f16 products, fp32 accumulation).  HA/HB pick the halves.
-template <int HA, int HB>
-__device__ __forceinline__ float hfma_f32(uint32_t a, uint32_t b, float c)
-{
-    float d;
-    if constexpr (HA == 0 && HB == 0)
-        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
-            "fma.rn.f32.f16 %0, a0, b0, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
-    else if constexpr (HA == 1 && HB == 0)
-        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
-            "fma.rn.f32.f16 %0, a1, b0, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
-    else if constexpr (HA == 0 && HB == 1)
-        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
-            "fma.rn.f32.f16 %0, a0, b1, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
-    else
-        asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
-            "fma.rn.f32.f16 %0, a1, b1, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
-    return d;
-}
-// Token weights are kept near 2^6 on the first group (room for the 2^8 of
-// softmax slack below the f16 limit) and scaled down when one would pass 2^15.
-constexpr int kVTargetExp = 6;
-constexpr float kVLimit = 32768.0f;
-
-// RoPE angles.  (sin a, cos a) of an fp32 angle 0 <= a < 2^17 * 2pi: a is
-// reduced modulo 2pi by the method of Cody and Waite ("Software Manual for the
-// Elementary Functions", 1980) with 2pi split in four parts, P1 = 101/16,
-// P2 = -15/512 and P3 = -75/2^22 of at most 7 significant bits (each k*P_i
-// exact in fp32 for k = rint(a/2pi) < 2^17, and each partial difference
-// exact) and P4 = fl(2pi - P1 - P2 - P3).  The reduced angle is within 2^-22
-// of the exact one; the hardware sine and cosine of it add at most 2^-21.4.
-// Positions are limited accordingly when a pre-RoPE cache is created.
-__device__ __forceinline__ void rope_sincos(float a, float *sn, float *cn)
-{
-    const float k = __fadd_rn(__fmaf_rn(a, 0.15915494f, 12582912.0f), -12582912.0f);
-    float r = __fmaf_rn(-k, 6.3125f, a);
-    r = __fmaf_rn(-k, -0.029296875f, r);
-    r = __fmaf_rn(-k, __uint_as_float(0xb7960000u), r);
-    r = __fmaf_rn(-k, __uint_as_float(0x338885a3u), r);
-    *sn = __sinf(r);
-    *cn = __cosf(r);
-}
-
-template <int DT>
-__device__ __forceinline__ float to_f(uint16_t b)
-{
-    if constexpr (DT == 1) return __uint_as_float((uint32_t)b << 16);
-    else return __half2float(__ushort_as_half(b));
-}
-__device__ __forceinline__ float f16f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
-
-__device__ __forceinline__ float warp_sum(float x)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
-    return x;
-}
-// Reduce-scatter of N per-lane values: at each level (lane offset OFF, OFF/2,
-// ...) a lane keeps half of its values and adds its partner's copy of them,
-// until one value is left, that of index h = the lane's bits OFF, OFF/2, ...
-// (most significant first), summed over those lanes.
-template <int N, int OFF>
-__device__ __forceinline__ float reduce_scatter(const float (&v)[N], int lane)
-{
-    if constexpr (N == 1) {
-        return v[0];
-    } else {
-        const bool up = lane & OFF;
-        float nv[N / 2];
-#pragma unroll
-        for (int i = 0; i < N / 2; ++i) {
-            const float keep = up ? v[N / 2 + i] : v[i];
-            const float send = up ? v[i] : v[N / 2 + i];
-            nv[i] = keep + __shfl_xor_sync(FULL, send, OFF);
-        }
-        return reduce_scatter<N / 2, OFF / 2>(nv, lane);
-    }
-}
-// out[h] = sum over the warp of v[h], for every h, in every lane (N a power
-// of two up to 16): a reduce-scatter, the rest of the butterfly, a gather.
-template <int N>
-__device__ __forceinline__ void warp_sum_n(const float (&v)[N], float (&out)[N], int lane)
-{
-    if constexpr (N == 1) {
-        out[0] = warp_sum(v[0]);
-    } else {
-        constexpr int LOG = N == 2 ? 1 : N == 4 ? 2 : N == 8 ? 3 : 4;
-        float x = reduce_scatter<N, 16>(v, lane);
-#pragma unroll
-        for (int o = 16 >> LOG; o > 0; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
-#pragma unroll
-        for (int h = 0; h < N; ++h) out[h] = __shfl_sync(FULL, x, h << (5 - LOG));
-    }
-}
-
-__device__ __forceinline__ float warp_max(float x)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(FULL, x, o));
-    return x;
-}
 
 // ---- shared-memory plan per warp ------------------------------------------------
 template <int D, int HG, bool ROPE>
@@ -314,8 +88,11 @@ struct WarpSmem {
     static constexpr int NST = ring_stages<HG, ROPE>();
     static constexpr int RING = 0;                  // NST x GB
     static constexpr int QP = NST * L::GB;          // float [HG][4][QPS]
+    static constexpr int PPF = 32 * HG + 4;                   // padded weight row (fp32), [token][head]
     static constexpr int PP = QP + HG * 4 * QPS * 4;          // f16 [HG][NJ][PPS]
-    static constexpr int QS = PP + (HG == 1 ? L::NJ * PPS * 2 : (HG / 2) * L::NJ * PPS2 * 4);  // float [HG][D]
+    static constexpr int PP_BYTES = values_f32<D, HG>() ? L::NJ * PPF * 4
+                                    : HG == 1 ? L::NJ * PPS * 2 : (HG / 2) * L::NJ * PPS2 * 4;
+    static constexpr int QS = PP + PP_BYTES;                  // float [HG][D]
     static constexpr int SZS = D / 4 + 4;                     // padded slice row (float2)
     static constexpr int SZ = QS + HG * D * 4;                // float2 [4][SZS] (RoPE)
     static constexpr int QRS = D / 8 + 2;                     // padded pair row (float2)
@@ -352,6 +129,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     constexpr int CPL = L::CPL, QPL = L::QPL, NJ = L::NJ, KW = L::KW, HALF = L::HALF, TPW = L::TPW;
     constexpr int PSTRIDE = D + 4;
     constexpr int kSt = W::NST;
+    constexpr bool VF32 = values_f32<D, HG>();
 
     extern __shared__ __align__(128) unsigned char smem_all[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -530,17 +308,18 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
             __syncwarp();
         }
         if (HG <= 2 && s < s_last) load_q(s + 1);
-        // The q'-writer lane's query channels, plain and with their pair-shift
-        // factors folded in (held in registers: measured faster than re-reading
-        // shared memory every group, even with four heads).
-        float qreg[HG][QPL], qsc[HG][QPL];
+        // The q'-writer lane's query channels: held in registers with one or
+        // two query heads per kv head (measured faster than re-reading shared
+        // memory every group); with four heads, where registers are short,
+        // re-read each group as one 16-byte load per head (QREG false).
+        constexpr bool QREG = HG <= 2;
+        float qreg[QREG ? HG : 1][QPL];
+        if constexpr (QREG) {
 #pragma unroll
-        for (int h = 0; h < HG; ++h)
+            for (int h = 0; h < HG; ++h)
 #pragma unroll
-            for (int e = 0; e < QPL; ++e) {
-                qreg[h][e] = qs[h * D + k_channel<D>(pcs, pL0 + e)];
-                qsc[h][e] = qreg[h][e] * (ROPE ? pair_scale(((pL0 + e) & 15) >> 1) : kq_scale(((pL0 + e) & 15) >> 1));
-            }
+                for (int e = 0; e < QPL; ++e) qreg[h][e] = qs[h * D + k_channel<D>(pcs, pL0 + e)];
+        }
 
         float m[HG], lsum[HG], zacc[HG][NJ];
         float2 accV[HG][CPL / 2];
@@ -596,21 +375,24 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                 const uint16_t *km = (const uint16_t *)(st + L::KM + lane * (D / 8));
                 float bias[HG];
                 if constexpr (!ROPE) {
+                    // Scales with their channel's code-pair factor folded in.
                     float sk[QPL], zk[QPL];
 #pragma unroll
                     for (int e = 0; e < QPL; ++e) {
-                        sk[e] = f16f(km[e]);
+                        sk[e] = f16f(km[e]) * kq_scale(((pL0 + e) & 15) >> 1);
                         zk[e] = f16f(km[QPL + e]);
                     }
                     float bp[HG];
 #pragma unroll
                     for (int h = 0; h < HG; ++h) {
                         bp[h] = 0.f;
-                        float qv[QPL];
+                        float qv[QPL], qh[QPL];
 #pragma unroll
                         for (int e = 0; e < QPL; ++e) {
-                            qv[e] = qsc[h][e] * sk[e];
-                            bp[h] = fmaf(qreg[h][e], zk[e], bp[h]);
+                            // (the lane's QPL channels are consecutive and 16-byte aligned)
+                            qh[e] = QREG ? qreg[QREG ? h : 0][e] : qs[h * D + k_channel<D>(pcs, pL0) + e];
+                            qv[e] = qh[e] * sk[e];
+                            bp[h] = fmaf(qh[e], zk[e], bp[h]);
                         }
                         float *dstq = qp + (h * 4 + pcs) * W::QPS + pL0;
 #pragma unroll
@@ -637,7 +419,46 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     kw[4 * c + 3] = v4.w;
                 }
                 float part[4][HG];
-                if constexpr (!ROPE) {
+                if constexpr (!ROPE && HG == 4 && KIVI_KEYS_SCALAR) {
+                    // Scalar FMAs: each query value stays the multiplicand of
+                    // four consecutive FMAs (one per token), which sustains
+                    // more multiply-adds per clock than fp32x2 FMAs whose
+                    // three operands all change (measured on B200).
+                    float accs[4][HG];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+#pragma unroll
+                        for (int h = 0; h < HG; ++h) accs[t][h] = 0.f;
+#pragma unroll
+                    for (int k = 0; k < KW; ++k) {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4) {
+                            // codes of local channels 16k + i + e, e = 0..3
+                            float c[4][4];
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const uint32_t w = kw[t * KW + k], w16 = w >> 16;
+                                c[t][0] = __uint_as_float(w & (3u << i));
+                                c[t][1] = __uint_as_float(w16 & (3u << i));
+                                c[t][2] = __uint_as_float(w & (12u << i));
+                                c[t][3] = __uint_as_float(w16 & (12u << i));
+                            }
+#pragma unroll
+                            for (int h = 0; h < HG; ++h) {
+                                const float4 q4 = *(const float4 *)(qp + (h * 4 + cs) * W::QPS + 16 * k + i);
+                                const float qe[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+#pragma unroll
+                                    for (int t = 0; t < 4; ++t) accs[t][h] = fmaf(qe[e], c[t][e], accs[t][h]);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+#pragma unroll
+                        for (int h = 0; h < HG; ++h) part[t][h] = accs[t][h];
+                } else if constexpr (!ROPE) {
                     float2 acc[4][HG];
 #pragma unroll
                     for (int t = 0; t < 4; ++t)
@@ -753,9 +574,21 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
 #pragma unroll
                     for (int h = 0; h < HG; ++h) zacc[h][j] = fmaf(pr[h], zvj, zacc[h][j]);
                 }
+                if constexpr (VF32) {
+                    // fp32 weights b[j][token][h] = p_h s_j 2^kVexp, one
+                    // 16-byte row entry per (group j, token) holding the heads.
+                    float ps[HG];
+#pragma unroll
+                    for (int h = 0; h < HG; ++h) ps[h] = pr[h] * pow2i(kVexp);
+                    float *ppf = (float *)pp;
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j)
+                        *(float4 *)(ppf + j * W::PPF + lane * HG) =
+                            make_float4(ps[0] * svj[j], ps[1] * svj[j], ps[2] * svj[j], ps[3] * svj[j]);
+                }
                 float fh[HG];
 #pragma unroll
-                for (int h = 0; h < HG; ++h) {
+                for (int h = 0; h < HG && !VF32; ++h) {
                     float f = pr[h] * evs[h];   // evs carries the lane's vtok
                     float bm = 0.f;
 #pragma unroll
@@ -785,7 +618,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     }
                     fh[h] = f;
                 }
-                if constexpr (HG == 1) {
+                if constexpr (VF32) {
+                } else if constexpr (HG == 1) {
 #pragma unroll
                     for (int j = 0; j < NJ; ++j)
                         pp[j * W::PPS + lane] = __half_as_ushort(__float2half_rn(fh[0] * svj[j]));
@@ -812,6 +646,30 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     vw[4 * c + 2] = v4.z;
                     vw[4 * c + 3] = v4.w;
                 }
+                if constexpr (VF32) {
+                    // Word u holds tokens A = 16vth + 2u (pairs 0..3, bits 2m
+                    // and 16 + 2m: channels 2m, 2m + 1 of the lane's octet)
+                    // and B = A + 1 (pairs 4..7, bits 8 + 2m and 24 + 2m).
+                    const float *ppf = (const float *)pp + jl * W::PPF + (16 * vth) * HG;
+#pragma unroll
+                    for (int u = 0; u < L::WPL; ++u) {
+                        const uint32_t w = vw[u], w8 = w >> 8, w16 = w >> 16, w24 = w >> 24;
+                        const float4 bA = *(const float4 *)(ppf + (2 * u) * HG);
+                        const float4 bB = *(const float4 *)(ppf + (2 * u + 1) * HG);
+                        const float wa[4] = {bA.x, bA.y, bA.z, bA.w}, wb[4] = {bB.x, bB.y, bB.z, bB.w};
+#pragma unroll
+                        for (int mm = 0; mm < CPL / 2; ++mm) {
+                            const uint32_t msk = 3u << (2 * mm);
+                            const float2 cA = make_float2(__uint_as_float(w & msk), __uint_as_float(w16 & msk));
+                            const float2 cB = make_float2(__uint_as_float(w8 & msk), __uint_as_float(w24 & msk));
+#pragma unroll
+                            for (int h = 0; h < HG; ++h) {
+                                accV[h][mm] = ffma2(make_float2(wa[h], wa[h]), cA, accV[h][mm]);
+                                accV[h][mm] = ffma2(make_float2(wb[h], wb[h]), cB, accV[h][mm]);
+                            }
+                        }
+                    }
+                } else {
                 // The weights of the lane's 16 tokens: one head, two tokens
                 // per word (HG == 1), or one token, two heads per word.
                 constexpr int PBW = HG == 1 ? 8 : 16;
@@ -855,6 +713,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                             }
                         }
                     }
+                }
                 }
             } else {
                 // ---------------- residual slice of up to 6 tokens ----------------
@@ -939,7 +798,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                     }
 #pragma unroll
                     for (int h = 0; h < HG; ++h) {
-                        const float pt = __shfl_sync(FULL, pr[h], 4 * (ok ? t : t0)) * pow2i(ev[h] - 24);
+                        const float pt = __shfl_sync(FULL, pr[h], 4 * (ok ? t : t0)) *
+                                         pow2i(VF32 ? kVexp - 149 : ev[h] - 24);
 #pragma unroll
                         for (int c = 0; c < CPL; c += 2) {
                             const float pa = pt * pow2i(c);   // 2^(2mm), mm = c/2
@@ -983,7 +843,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
 #pragma unroll
             for (int c = 0; c < CPL; c += 2) {
                 const float2 a = accV[h][c / 2];
-                const float f = pow2i(24 - c - ev[h]);   // 2^(24 - 2mm - ev)
+                // 2^(24 - 2mm - ev), or 2^(149 - kVexp - 2mm) for fp32 weights
+                const float f = pow2i(VF32 ? 149 - kVexp - c : 24 - c - ev[h]);
                 const float x = a.x + __shfl_xor_sync(FULL, a.x, 16);
                 const float y = a.y + __shfl_xor_sync(FULL, a.y, 16);
                 o[h][c] = fmaf(x, f, zt[h]);
