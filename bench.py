@@ -132,6 +132,19 @@ def decode_bytes(w, n_q, r):
     return w.B * w.H_kv * (n_q * per_q + r * per_r) + w.B * w.H_q * w.D * (2 + 4)
 
 
+def decode_flops(w, n_q, r):
+    """Algorithmic flops of one decode call: per (token, query head) a D-long
+    dot product with the key and a D-long weighted sum of the value, 2 flops
+    per multiply-add each."""
+    return 4 * w.D * w.B * w.H_q * (n_q + r)
+
+
+def fma_peak_tflops(sms, sm_mhz):
+    """fp32 FMA peak of the CUDA cores: 4 schedulers per SM, each issuing one
+    32-lane FMA instruction per clock (2 flops per lane)."""
+    return sms * 4 * 32 * 2 * sm_mhz * 1e6 / 1e12
+
+
 def fused_append_bytes(w):
     """A fused launch also reads k_t, v_t and writes them to the residual."""
     return 4 * w.B * w.H_kv * w.D * 2
@@ -481,6 +494,8 @@ class Workbench:
                    for row in self.steps]
         self.Op = [ctypes.c_void_p(o.data_ptr()) for o in self.outs]
         self.units_step = sum(decode_units(w, n, r) for n, r, _ in self.calls) * layers
+        self.flops_step = sum(decode_flops(w, n, r) for n, r, _ in self.calls) * layers
+        self.sms = torch.cuda.get_device_properties(dev).multi_processor_count
         self.bytes_step = (sum(decode_bytes(w, n, r) for n, r, _ in self.calls)
                            + fused_append_bytes(w) * sum(k == "fused" for _, _, k in self.calls)) * layers
         self.n_dec = layers * len(self.calls)
@@ -553,6 +568,39 @@ class Workbench:
             c.close()
 
 
+def sm_clock(t):
+    """Median SM clock sampled during the timed region (MHz), else the B200's
+    maximum."""
+    ck = t.get("clocks") or {}
+    return ck.get("sm_mhz") or ck.get("sm_max_mhz") or 1965.0
+
+
+def roofline(wb, dec_avg_ms, t, peak, peak_kind, traffic):
+    """The decode kernel against both ceilings that can bind it: HBM (its
+    algorithmic bytes per launch over the measured copy bandwidth) and the
+    CUDA cores' fp32 FMA peak (its algorithmic flops per launch).  `bound`
+    names the one it is closer to; the other is reported beside it."""
+    bpl = wb.bytes_step / wb.n_dec
+    fpl = wb.flops_step / wb.n_dec
+    gbs = bpl / (dec_avg_ms / 1e3) / 1e9
+    tfs = fpl / (dec_avg_ms / 1e3) / 1e12
+    mhz = sm_clock(t)
+    fpk = fma_peak_tflops(wb.sms, mhz)
+    hbm = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+           "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+           "alg_bytes_per_launch": bpl, "frac_of_8TBps": gbs / 8000.0}
+    alu = {"bound": "alu", "achieved": tfs, "peak": fpk, "unit": "TFLOP/s", "frac": tfs / fpk,
+           "peak_source": (f"fp32 FMA peak of the CUDA cores: {wb.sms} SMs x 128 FMA/clk x 2 flops "
+                           f"x {mhz:.0f} MHz (median SM clock sampled in the timed region)"),
+           "alg_flops_per_launch": fpl}
+    main, other = (alu, hbm) if alu["frac"] > hbm["frac"] else (hbm, alu)
+    out = dict(main)
+    out["traffic"] = traffic
+    out["kernel"] = "decode_kernel (kivi_decode_attn / kivi_append_decode)"
+    out["other_bound"] = other
+    return out
+
+
 def summarize(wb, t, steps, world, peak):
     """Per-workload figures from a Workbench measurement."""
     w = wb.w
@@ -560,6 +608,9 @@ def summarize(wb, t, steps, world, peak):
     pre_avg = sum(t["pre_ms"]) / len(t["pre_ms"])
     bpl = wb.bytes_step / wb.n_dec
     achieved = bpl / (dec_avg / 1e3) / 1e9
+    fpl = wb.flops_step / wb.n_dec
+    tfs = fpl / (dec_avg / 1e3) / 1e12
+    fpk = fma_peak_tflops(wb.sms, sm_clock(t))
     pb = prefill_bytes(w)
     return {
         "value": world * wb.units_step * steps / (t["ms"] / 1e3), "unit": UNIT,
@@ -569,6 +620,8 @@ def summarize(wb, t, steps, world, peak):
                    "launches_timed": len(t["dec_ms"]), "alg_bytes_per_launch": bpl,
                    "achieved_gbs": achieved, "frac_of_measured_hbm": achieved / peak,
                    "frac_of_8TBps": achieved / 8000.0,
+                   "alg_flops_per_launch": fpl, "achieved_tflops": tfs,
+                   "frac_of_fma_peak": tfs / fpk,
                    "tokens_heads_per_s": wb.units_step / wb.n_dec / (dec_avg / 1e3),
                    "gpu_time_share": sum(t["dec_ms"]) / t["ms"]},
         "prefill": {"avg_us": 1e3 * pre_avg, "alg_bytes": pb,
@@ -633,7 +686,8 @@ def run_gpu(args):
     dec_avg = reduce_max(sum(t["dec_ms"]) / len(t["dec_ms"]), dev)
     t["ms"] = ms
     s = summarize(wb, t, args.steps, world, peak)
-    achieved = s["decode"]["alg_bytes_per_launch"] / (dec_avg / 1e3) / 1e9
+    roof = roofline(wb, dec_avg, t, peak, peak_kind,
+                    traffic_per_launch(w, not (args.batch or args.decode_steps)))
     e2e = run_e2e(args, wb, world) if sets == layers else None
     launches = wb.launches_step * args.steps
     wb.close()
@@ -652,13 +706,7 @@ def run_gpu(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
             "data": "synthetic", "config": workload_config(w, args, layers, world, sets),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak,
-                         "traffic": traffic_per_launch(w, not (args.batch or args.decode_steps)),
-                         "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                         "kernel": "decode_kernel (kivi_decode_attn / kivi_append_decode)",
-                         "alg_bytes_per_launch": s["decode"]["alg_bytes_per_launch"],
-                         "frac_of_8TBps": achieved / 8000.0},
+            "roofline": roof,
             "decode_attn": s["decode"], "prefill": s["prefill"],
             "e2e": e2e, "gpu_launches": launches, "clocks": s["clocks"],
             "cpu_baseline": cpu, "per_config": per_config,

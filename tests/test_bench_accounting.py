@@ -105,3 +105,31 @@ def test_oracle_sample_units():
     one, calls, units = bench.oracle_sample(w, 8)
     assert (one.B, one.H_kv, one.H_q) == (1, 1, 4) and len(calls) == 8
     assert units == sum(n + r for n, r, _ in bench.decode_calls(w)[:8])
+
+
+def test_decode_flops_and_fma_peak():
+    w = W["mistral_gqa"]
+    # 4*D flops per (token, query head): 64 x 32 query heads x 32,769 tokens
+    assert bench.decode_flops(w, 32768, 1) == 4 * 128 * 64 * 32 * 32769
+    # 148 SMs x 4 schedulers x 32 lanes x 2 flops at 1,965 MHz
+    assert abs(bench.fma_peak_tflops(148, 1965.0) - 74.4499) < 1e-3
+
+
+def test_roofline_names_the_closer_bound():
+    import types
+    w = W["mistral_gqa"]
+    n_q, r = 32768, 1
+    wb = types.SimpleNamespace(bytes_step=bench.decode_bytes(w, n_q, r), n_dec=1,
+                               flops_step=bench.decode_flops(w, n_q, r), sms=148)
+    t = {"clocks": {"sm_mhz": 1965.0}}
+    # at 930 us: ~1.69 TB/s (26% of 6,454 GB/s) but ~36.9 TFLOP/s (50% of 74.4)
+    roof = bench.roofline(wb, 0.930, t, 6454.3, "measured", None)
+    assert roof["bound"] == "alu" and roof["unit"] == "TFLOP/s"
+    assert 0.49 < roof["frac"] < 0.51 and roof["other_bound"]["bound"] == "hbm"
+    assert 0.25 < roof["other_bound"]["frac"] < 0.27
+    # one query head per kv head at the MHA layer's 38 us: HBM is the closer bound
+    w2 = W["llama2_7b_layer"]
+    wb2 = types.SimpleNamespace(bytes_step=bench.decode_bytes(w2, 4096, 1), n_dec=1,
+                                flops_step=bench.decode_flops(w2, 4096, 1), sms=148)
+    roof2 = bench.roofline(wb2, 0.038, t, 6454.3, "measured", 1.0)
+    assert roof2["bound"] == "hbm" and roof2["traffic"] == 1.0 and roof2["other_bound"]["bound"] == "alu"
