@@ -83,6 +83,7 @@ def lib():
     L.kivi_cache_bytes.argtypes = [vp, P(_Bytes)]
     L.kivi_export.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp]
     L.kivi_device_status.argtypes = [vp, P(i32)]
+    L.kivi_debug_expire_first_wait.argtypes = [vp, i32]
     L.kivi_cache_destroy.argtypes = [vp]
     L.kivi_decode_split.argtypes = [i64, i64, i32, i32, i32, i64, i64, i64, P(i64)]
     L.kivi_fake_quant.argtypes = [vp, i32, i64, i64, i32, i32, i32, i32, i32, i32, vp, vp, vp]
@@ -91,7 +92,8 @@ def lib():
                  "kivi_append_decode",
                  "kivi_cache_reset",
                  "kivi_cache_length", "kivi_cache_bytes", "kivi_export", "kivi_device_status",
-                 "kivi_cache_destroy", "kivi_decode_split", "kivi_fake_quant"):
+                 "kivi_debug_expire_first_wait", "kivi_cache_destroy", "kivi_decode_split",
+                 "kivi_fake_quant"):
         getattr(L, name).restype = st
     _lib = L
     return L
@@ -248,6 +250,11 @@ class KiviCache:
         b = _Bytes()
         _check(lib().kivi_cache_bytes(self._h, ctypes.byref(b)), "kivi_cache_bytes")
         return {f: getattr(b, f) for f, _ in _Bytes._fields_}
+
+    def debug_expire_first_wait(self, on: bool = True):
+        """Testing the failure path: later decode launches have each warp's
+        first wait give up at once (see kivi_debug_expire_first_wait)."""
+        _check(lib().kivi_debug_expire_first_wait(self._h, int(on)), "kivi_debug_expire_first_wait")
 
     def device_status(self) -> int:
         code = ctypes.c_int()

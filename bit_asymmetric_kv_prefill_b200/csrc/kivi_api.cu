@@ -111,6 +111,7 @@ struct kivi_cache {
     int r;
     bool prefilled;
     int wg, wr;
+    int expire_first_wait;   // testing only (kivi_debug_expire_first_wait)
 };
 
 namespace {
@@ -210,6 +211,7 @@ kivi_status kivi_cache_create_ex(const kivi_config *cfg, kivi_cache **out)
     c->n_q = 0;
     c->r = 0;
     c->prefilled = false;
+    c->expire_first_wait = 0;
     c->wg = env_int("KIVI_SPLIT_WG", 4);
     c->wr = env_int("KIVI_SPLIT_WR", 3);
     *out = c;
@@ -385,6 +387,13 @@ kivi_status kivi_decode_attn(kivi_cache *c, const void *q, int H_q, float *out, 
     p.slots = c->plan.slots;
     cudaError_t e = launch_decode(D, HG, dtype, pre_rope, p, (cudaStream_t)stream);
     return cuda_status(e);
+}
+
+kivi_status kivi_debug_expire_first_wait(kivi_cache *c, int on)
+{
+    if (!c) return KIVI_ERR_ARG;
+    c->expire_first_wait = on ? 1 : 0;
+    return KIVI_OK;
 }
 
 kivi_status kivi_device_status(kivi_cache *c, int *code)
@@ -576,6 +585,7 @@ kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q
     p->inv_freq = c->inv_freq;
     p->newK = p->newV = nullptr;
     p->new_slot = -1;
+    p->expire_first_wait = c->expire_first_wait;
     p->magic = 0x4B000000u;
     p->neg_magic = -8388608.0f;
     *D = c->cfg.D;

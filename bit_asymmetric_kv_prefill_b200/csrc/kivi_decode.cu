@@ -250,9 +250,13 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     for (int i = 0; i < kSt; ++i) issue_next();
 
     bool failed = false;
+    // Bounded wait for the next stage.  With p.expire_first_wait (testing the
+    // failure path) the warp's first consuming wait gives up at once; every
+    // later wait, the drain's included, keeps the full bound.
     auto wait_stage = [&]() -> bool {
         const uint32_t bar = bar0 + 8 * cst;
-        for (int it = 0; it < kWaitLimit; ++it)
+        const int limit = (p.expire_first_wait && consumed == 0 && !failed) ? 0 : kWaitLimit;
+        for (int it = 0; it < limit; ++it)
             if (__all_sync(FULL, mbar_try_wait(bar, cph))) return true;
         return false;
     };

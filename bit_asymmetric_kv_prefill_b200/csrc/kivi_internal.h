@@ -57,6 +57,9 @@ struct DecodeParams {
     // newV ([seqs][D]) and stored to the residual by the decode (else null, -1).
     const uint16_t *newK, *newV;
     int new_slot;
+    // Testing the failure path: each warp's first consuming wait gives up at
+    // once (the kernel then reports a failed wait and drains its copies).
+    int expire_first_wait;
 };
 
 int num_sms();

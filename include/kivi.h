@@ -203,6 +203,22 @@ KIVI_API kivi_status kivi_export(const kivi_cache *c, long long seq0, long long 
  * bounded wait in its kernels completed, else the code of the first failure. */
 KIVI_API kivi_status kivi_device_status(kivi_cache *c, int *code);
 
+/* Testing the failure path (no part of the method corresponds to this call):
+ * with on != 0, every later decode launch on c (kivi_decode_attn,
+ * kivi_append_decode, kivi_decode_attn_noalloc) has each warp's first wait
+ * for its staged data give up at once.  The warps then record
+ * KIVI_DEVICE_WAIT_TIMEOUT in the status word, let the copies they issued
+ * land (those waits keep their full bound) and return without writing their
+ * results, so `out` is undefined, and a fused append may not have stored its
+ * token: as after any device-side failure, reset and prefill the cache again
+ * before relying on its contents.  kivi_device_status reports and clears the
+ * failure; with on = 0 the next launch runs normally.  Nothing faults or
+ * hangs. */
+KIVI_API kivi_status kivi_debug_expire_first_wait(kivi_cache *c, int on);
+
+/* Status word value recorded when a bounded wait in a kernel gave up. */
+#define KIVI_DEVICE_WAIT_TIMEOUT 1
+
 /* Release the cache (frees its memory unless it lives in a caller workspace). */
 KIVI_API kivi_status kivi_cache_destroy(kivi_cache *c);
 

@@ -328,6 +328,45 @@ def test_calls_with_another_device_current_are_refused():
     assert c.length() == (0, 41) and c.device_status() == 0
 
 
+EXPIRE = [("llama2_7b_layer", dict(B=2, H_q=2, H_kv=2, T=700), False),
+          ("mistral_gqa", dict(B=3, H_q=8, H_kv=2, T=1500), True),
+          ("long_context", dict(B=1, H_q=8, H_kv=2, T=400), True)]
+
+
+@pytest.mark.parametrize("name,kw,fused", EXPIRE, ids=[n for n, _, _ in EXPIRE])
+def test_an_expired_wait_is_reported_and_the_next_call_is_clean(name, kw, fused):
+    """A decode whose warps' first waits give up (the test switch) reports the
+    failed wait in the status word without faulting or hanging; reading the
+    status clears it, and the next call gives the normal result bit for bit."""
+    w = small(name, steps=2, **kw)
+    K, V = synth.prefill_inputs(w, 12, device=DEV)
+    k, v, q = synth.step_inputs(w, 1, 12, device=DEV)
+    mk = lambda: KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, w.T_max,
+                           pre_rope=w.pre_rope, rope_theta=w.rope_theta)
+    a, c = mk(), mk()
+    for x in (a, c):
+        x.prefill(K, V)
+    ref = a.append_decode(k, v, q) if fused else a.decode(q)
+    c.debug_expire_first_wait(True)
+    if fused:
+        c.append_decode(k, v, q)
+    else:
+        c.decode(q)
+    torch.cuda.synchronize()
+    assert c.device_status() == 1            # KIVI_DEVICE_WAIT_TIMEOUT
+    assert c.device_status() == 0            # read and cleared
+    c.debug_expire_first_wait(False)
+    if fused:
+        # the failed launch may not have stored its token: start the cache over
+        c.reset()
+        c.prefill(K, V)
+        assert torch.equal(c.append_decode(k, v, q), ref)
+    else:
+        assert torch.equal(c.decode(q), ref)
+    assert torch.equal(c.decode(q), a.decode(q))
+    assert c.device_status() == 0 and a.device_status() == 0
+
+
 def test_caller_workspace_holds_the_whole_cache():
     w = small("tiny", T=300, B=2, steps=0)
     n = KiviCache.required_bytes(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, 300)
