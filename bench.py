@@ -902,7 +902,33 @@ def run_diag(args):
         for which, axis, sym, sparse in (("K", ka, ks, ko), ("V", va, vs, vo)):
             launch(which, axis, sym, sparse, values=False)
             modes[mode][f"{which}_rel_err"] = (float(err.sum()) / norms[which]) ** 0.5
-    launches = len(plan) * args.steps
+    # Non-uniform levels (KVQuant's non-uniform quantization): four levels
+    # fitted by Lloyd's algorithm on a few matrices of the same cache (keys per
+    # channel, values per token), timed like the modes above.
+    from oracle import diag as odiag
+    nuq = {}
+    for which, axis in (("K", 0), ("V", 1)):
+        Xs = (K if which == "K" else V).reshape(N, T, D)
+        lev = odiag.fit_levels(Xs[:2].float().cpu().numpy(), axis, 32, 4)
+        levc = (ctypes.c_double * 4)(*[float(v) for v in lev])
+        run = lambda: L.kivi_fake_quant_levels(src[which], dt, N, T, D, axis, 32, 4, levc, xhp, None,
+                                               errp, sp)
+        for _ in range(args.warmup):
+            if run():
+                raise RuntimeError("kivi_fake_quant_levels failed")
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            run()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        us = 1e3 * e0.elapsed_time(e1) / args.steps
+        nuq[f"{which}_us"] = us
+        nuq[f"{which}_gbs"] = elems * 6 / (us / 1e6) / 1e9
+        nuq[f"{which}_rel_err"] = (float(err.sum()) / norms[which]) ** 0.5
+        nuq[f"{which}_levels"] = [float(v) for v in lev]
+    modes["nonuniform_levels_4"] = nuq
+    launches = len(plan) * args.steps + 2 * args.steps
     cpu = None
     if not args.no_cpu_baseline:
         # the oracle as it stands, single-threaded, on whole key matrices of

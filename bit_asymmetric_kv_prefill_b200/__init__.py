@@ -87,13 +87,15 @@ def lib():
     L.kivi_cache_destroy.argtypes = [vp]
     L.kivi_decode_split.argtypes = [i64, i64, i32, i32, i32, i64, i64, i64, P(i64)]
     L.kivi_fake_quant.argtypes = [vp, i32, i64, i64, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+    L.kivi_fake_quant_levels.argtypes = [vp, i32, i64, i64, i32, i32, i32, i32, P(ctypes.c_double),
+                                         vp, vp, vp, vp]
     for name in ("kivi_cache_create", "kivi_cache_create_ex", "kivi_cache_required_bytes",
                  "kivi_prefill", "kivi_append", "kivi_decode_attn", "kivi_decode_attn_noalloc",
                  "kivi_append_decode",
                  "kivi_cache_reset",
                  "kivi_cache_length", "kivi_cache_bytes", "kivi_export", "kivi_device_status",
                  "kivi_debug_expire_first_wait", "kivi_cache_destroy", "kivi_decode_split",
-                 "kivi_fake_quant"):
+                 "kivi_fake_quant", "kivi_fake_quant_levels"):
         getattr(L, name).restype = st
     _lib = L
     return L
@@ -323,3 +325,32 @@ def fake_quant(x: torch.Tensor, axis: int, G: int = 32, bits: int = 2, symmetric
                                  err.data_ptr() if err is not None else None, _stream_ptr(stream)),
            "kivi_fake_quant")
     return xh, err
+
+
+def fake_quant_levels(x: torch.Tensor, axis: int, G: int, levels, values: bool = True,
+                      codes: bool = False, error: bool = True, stream=None):
+    """Quantize-dequantize every [T, D] matrix of x ([..., T, D], bf16 or fp16,
+    on the GPU) with non-uniform levels per group (see kivi_fake_quant_levels):
+    each group's elements are coded by the nearest of the normalized
+    ``levels`` on the group's [min, max].
+
+    Returns (x_hat, codes, sq_err): x_hat fp32 with x's shape, codes uint8 with
+    x's shape, sq_err fp64 [prod(leading dims)]; each None unless asked for."""
+    if not isinstance(x, torch.Tensor) or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA tensor")
+    if x.dim() < 2:
+        raise ValueError("x must have shape [..., T, D]")
+    T, D = x.shape[-2], x.shape[-1]
+    N = x.numel() // max(T * D, 1)
+    lev = (ctypes.c_double * len(levels))(*[float(v) for v in levels])
+    xh = torch.empty(x.shape, dtype=torch.float32, device=x.device) if values else None
+    cc = torch.empty(x.shape, dtype=torch.uint8, device=x.device) if codes else None
+    err = torch.empty(N, dtype=torch.float64, device=x.device) if error else None
+    _check(lib().kivi_fake_quant_levels(x.data_ptr(), _dtype_code(x.dtype), N, T, D, axis, G,
+                                        len(levels), lev,
+                                        xh.data_ptr() if xh is not None else None,
+                                        cc.data_ptr() if cc is not None else None,
+                                        err.data_ptr() if err is not None else None,
+                                        _stream_ptr(stream)),
+           "kivi_fake_quant_levels")
+    return xh, cc, err

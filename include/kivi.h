@@ -280,6 +280,31 @@ KIVI_API kivi_status kivi_fake_quant(const void *x, kivi_dtype dtype, long long 
                                      int D, int axis, int G, int bits, int symmetric,
                                      int outlier, float *xhat, double *sq_err, void *stream);
 
+/*
+ * Diagnostic quantization with non-uniform levels per group (KVQuant summary,
+ * "Non-Uniform KV Cache Quantization"; the pages give only the name).  Every
+ * group (axis and G as in kivi_fake_quant, any G >= 1 dividing T per channel
+ * or D per token) keeps its minimum and maximum (fp32) and codes each element
+ * by the nearest of nlev normalized levels on [min, max]:
+ *   u = (x - min) / (max - min)               IEEE fp64 subtract and divide
+ *   code = argmin_k |u - levels[k]|           the first level on ties
+ *   x_hat = fp32(min + (max - min) * levels[code])   fp64 multiply, then add
+ * A group with max == min decodes to its value with code 0.  It touches no
+ * cache.
+ *   x       DEVICE [N, T, D] in `dtype`, 16-byte aligned.
+ *   levels  HOST array of nlev doubles in [0, 1] (any order), 2 <= nlev <= 256;
+ *           copied into the launch.
+ *   xhat    DEVICE [N, T, D] fp32, 16-byte aligned, or NULL.
+ *   codes   DEVICE [N, T, D] uint8, or NULL.
+ *   sq_err  DEVICE [N] fp64, 8-byte aligned, or NULL: sum over each matrix of
+ *           (x - x_hat)^2 in fp64 (summation order unspecified).
+ * At least one output is non-NULL.  Asynchronous on `stream`; KIVI_ERR_ARG for
+ * bad pointers, sizes, levels or alignment.
+ */
+KIVI_API kivi_status kivi_fake_quant_levels(const void *x, kivi_dtype dtype, long long N, long long T,
+                                            int D, int axis, int G, int nlev, const double *levels,
+                                            float *xhat, uint8_t *codes, double *sq_err, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -178,3 +178,93 @@ def test_full_size_llama2_13b_layer_sampled(axis, bits, sym):
             got = xh_flat[n].cpu().numpy()
             assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
         del xh, err, d
+
+
+# ---- non-uniform levels (kivi_fake_quant_levels) ----------------------------------
+
+def check_levels(x, axis, G, levels):
+    """GPU non-uniform levels on x against oracle_fake_quant_levels: x_hat and
+    codes bit-exact (both sides evaluate the same IEEE fp64 operations), the
+    per-matrix squared error against float64 within summation-order rounding."""
+    xh, cc, err = kv.fake_quant_levels(x, axis, G, levels, codes=True)
+    torch.cuda.synchronize()
+    xf = x.float().cpu().numpy()
+    ref, rc = oracle.fake_quant_levels(xf, axis, G, levels, codes=True)
+    got = xh.cpu().numpy()
+    bad = got.view(np.uint32) != ref.view(np.uint32)
+    assert not bad.any(), (f"{bad.sum()} x_hat mismatches, first at {np.argwhere(bad)[0]}: "
+                           f"{got[bad][0]!r} vs {ref[bad][0]!r}")
+    np.testing.assert_array_equal(cc.cpu().numpy().astype(np.int32), rc)
+    T, D = x.shape[-2:]
+    d = (xf.astype(np.float64) - ref.astype(np.float64)).reshape(-1, T * D)
+    np.testing.assert_allclose(err.cpu().numpy(), (d * d).sum(axis=1), rtol=1e-12, atol=1e-300)
+
+
+LEVELS = [[0.0, 1 / 3, 2 / 3, 1.0], [0.0, 0.1, 0.35, 0.9], [0.05, 0.5, 0.95], [0.9, 0.1, 0.5, 0.0],
+          [0.0, 1.0], list(np.linspace(0.0, 1.0, 16)), list(np.sort(np.random.default_rng(3).random(256)))]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("axis", [PC, PT])
+@pytest.mark.parametrize("li", range(len(LEVELS)), ids=[f"lev{len(l)}-{i}" for i, l in enumerate(LEVELS)])
+def test_levels_match_oracle(dtype, axis, li):
+    K, V = recipe("llama2_7b_layer", H=3, T=352, dtype=dtype, seed=li)
+    for x in (K, V):
+        check_levels(x, axis, 32, LEVELS[li])
+
+
+@pytest.mark.parametrize("axis,G", [(PC, 1), (PC, 7), (PC, 11), (PT, 1), (PT, 3), (PT, 64), (PT, 128)])
+def test_levels_group_sizes(axis, G):
+    T = 77 if axis == PC else 50
+    D = 4 * G if axis == PT else 48
+    x = (torch.randn(2, T - T % G if axis == PC else T, D, generator=torch.Generator().manual_seed(G)) * 3)
+    check_levels(x.to(torch.bfloat16).cuda(), axis, G, [0.0, 0.2, 0.45, 1.0])
+
+
+def test_levels_ties_grids_and_constant_groups():
+    # values on the level grid come back exactly; points halfway between two
+    # levels take the first of them; constant groups keep their value
+    g = torch.Generator().manual_seed(5)
+    T, D = 64, 32
+    lev = [0.0, 0.25, 0.5, 1.0]
+    base = torch.randint(-8, 8, (T, D), generator=g).float()
+    pick = torch.tensor(lev)[torch.randint(0, 4, (T, D), generator=g)]
+    x = base + 8.0 * pick
+    x[0:32:2, :] = base[0:32:2, :]                      # each group holds its min ...
+    x[1:32:2, :] = base[1:32:2, :] + 8.0                # ... and its max
+    x[32:64, 3] = 2.5                                   # constant groups
+    x[40, 5] = x[32:64, 5].min() + 0.375 * (x[32:64, 5].max() - x[32:64, 5].min())  # tie 0.25 / 0.5
+    for dt in (torch.bfloat16, torch.float16):
+        check_levels(x.to(dt).cuda()[None], PC, 32, lev)
+        check_levels(x.t().contiguous().to(dt).cuda()[None], PT, 32, lev)
+
+
+def test_levels_rejects_bad_arguments():
+    x = torch.zeros(1, 64, 32, dtype=torch.bfloat16, device="cuda")
+    for axis, G, lev in [(PC, 32, [0.0]), (PC, 32, [0.0, 1.5]), (PC, 32, [float("nan"), 0.5]),
+                         (PC, 30, [0.0, 1.0]), (PT, 5, [0.0, 1.0]), (PC, 32, [0.0] * 257)]:
+        with pytest.raises(kv.KiviError) as e:
+            kv.fake_quant_levels(x, axis, G, lev)
+        assert e.value.code == 1
+
+
+@pytest.mark.parametrize("axis", [PC, PT])
+def test_levels_full_size_llama2_13b_layer_sampled(axis):
+    """One full Llama-2-13B layer cache (16 x 40 heads x 4,096 tokens x 128):
+    four levels fitted to its keys by Lloyd's algorithm (the oracle's fitting),
+    sampled matrices checked one by one and every matrix's error against the
+    values the launch returns."""
+    from oracle import diag
+    w = synth.WORKLOADS["llama2_13b_cache"]
+    K, V = synth.prefill_inputs(w, seed=2, device="cuda")
+    N, T, D = w.B * w.H_kv, w.T, w.D
+    Kn = K.reshape(N, T, D)
+    lev = diag.fit_levels(Kn[:4].float().cpu().numpy(), axis, 32, 4)
+    xh, cc, err = kv.fake_quant_levels(Kn, axis, 32, lev, codes=True)
+    torch.cuda.synchronize()
+    for i in (0, 217, N - 1):
+        ref, rc = oracle.fake_quant_levels(Kn[i].float().cpu().numpy(), axis, 32, lev, codes=True)
+        assert np.array_equal(xh[i].cpu().numpy().view(np.uint32), ref.view(np.uint32)), i
+        assert np.array_equal(cc[i].cpu().numpy().astype(np.int32), rc), i
+    own = (Kn.double() - xh.double()).pow(2).sum(dim=(1, 2))
+    torch.testing.assert_close(err, own, rtol=1e-12, atol=0)
