@@ -74,6 +74,8 @@ def lib():
     L.kivi_cache_create_ex.argtypes = [P(_Config), P(vp)]
     L.kivi_cache_required_bytes.argtypes = [P(_Config), P(ctypes.c_size_t)]
     L.kivi_prefill.argtypes = [vp, vp, vp, i64, vp]
+    L.kivi_prefill_ragged.argtypes = [vp, vp, vp, i64, P(i64), vp]
+    L.kivi_cache_length_at.argtypes = [vp, i32, P(i64), P(i32)]
     L.kivi_append.argtypes = [vp, vp, vp, vp]
     L.kivi_decode_attn.argtypes = [vp, vp, i32, vp, vp]
     L.kivi_append_decode.argtypes = [vp, vp, vp, vp, i32, vp, vp]
@@ -90,7 +92,7 @@ def lib():
     L.kivi_fake_quant_levels.argtypes = [vp, i32, i64, i64, i32, i32, i32, i32, P(ctypes.c_double),
                                          vp, vp, vp, vp]
     for name in ("kivi_cache_create", "kivi_cache_create_ex", "kivi_cache_required_bytes",
-                 "kivi_prefill", "kivi_append", "kivi_decode_attn", "kivi_decode_attn_noalloc",
+                 "kivi_prefill", "kivi_prefill_ragged", "kivi_cache_length_at", "kivi_append", "kivi_decode_attn", "kivi_decode_attn_noalloc",
                  "kivi_append_decode",
                  "kivi_cache_reset",
                  "kivi_cache_length", "kivi_cache_bytes", "kivi_export", "kivi_device_status",
@@ -193,6 +195,17 @@ class KiviCache:
         _check(lib().kivi_prefill(self._h, self._tensor(K, shape, "K"), self._tensor(V, shape, "V"),
                                   T, _stream_ptr(stream)), "kivi_prefill")
 
+    def prefill_ragged(self, K: torch.Tensor, V: torch.Tensor, lengths, stream=None):
+        """Prefill with batch element b holding its first lengths[b] tokens of
+        K, V [B, H_kv, T_pad, D] (see kivi_prefill_ragged)."""
+        T_pad = K.shape[2]
+        shape = (self.B, self.H_kv, T_pad, self.D)
+        if len(lengths) != self.B:
+            raise ValueError(f"lengths must hold {self.B} values")
+        arr = (ctypes.c_longlong * self.B)(*[int(t) for t in lengths])
+        _check(lib().kivi_prefill_ragged(self._h, self._tensor(K, shape, "K"), self._tensor(V, shape, "V"),
+                                         T_pad, arr, _stream_ptr(stream)), "kivi_prefill_ragged")
+
     def append(self, k: torch.Tensor, v: torch.Tensor, stream=None):
         shape = (self.B, self.H_kv, self.D)
         _check(lib().kivi_append(self._h, self._tensor(k, shape, "k_t"), self._tensor(v, shape, "v_t"),
@@ -248,6 +261,13 @@ class KiviCache:
                "kivi_cache_length")
         return n_q.value, r.value
 
+    def length_at(self, b: int):
+        """(n_q, r) of batch element b."""
+        n_q, r = ctypes.c_longlong(), ctypes.c_int()
+        _check(lib().kivi_cache_length_at(self._h, b, ctypes.byref(n_q), ctypes.byref(r)),
+               "kivi_cache_length_at")
+        return n_q.value, r.value
+
     def nbytes(self) -> dict:
         b = _Bytes()
         _check(lib().kivi_cache_bytes(self._h, ctypes.byref(b)), "kivi_cache_bytes")
@@ -268,7 +288,7 @@ class KiviCache:
         [seq0, seq0 + nseq), sequence = b*H_kv + h."""
         import numpy as np
         nseq = self.B * self.H_kv - seq0 if nseq is None else nseq
-        n_q, r = self.length()
+        n_q, r = self.length_at(seq0 // self.H_kv)   # the range shares one split
         D, G = self.D, self.G
         a = dict(codesK=np.zeros((nseq, n_q, D), np.uint8), codesV=np.zeros((nseq, n_q, D), np.uint8),
                  sK=np.zeros((nseq, n_q // G, D), np.uint16), zK=np.zeros((nseq, n_q // G, D), np.uint16),

@@ -26,7 +26,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Plan {
     long long seqs, ngcap;
-    int slots;
+    long long part_rows;   // decode partial rows: every split has at most warps + seqs
     size_t off_packed, off_resK, off_resV, off_part, off_tick, off_err, off_freq, total;
     size_t codes, meta, residual, scratch;
 };
@@ -50,11 +50,11 @@ kivi_status make_plan(const kivi_config *c, int sms, Plan *p)
     p->seqs = (long long)c->B * c->H_kv;
     p->ngcap = (c->T_max + c->G - 1) / c->G;
     const long long max_warps = (long long)sms * kMaxWarpsPerCta;
-    p->slots = (int)(max_warps / p->seqs + 2);
+    p->part_rows = max_warps + p->seqs;
     const size_t gb = (size_t)24 * c->D;
     const size_t packed = (size_t)p->seqs * p->ngcap * gb;
     const size_t res = (size_t)p->seqs * c->R * c->D * 2;
-    const size_t part = (size_t)p->seqs * p->slots * kMaxGroupHeads * (c->D + 4) * sizeof(float);
+    const size_t part = (size_t)p->part_rows * kMaxGroupHeads * (c->D + 4) * sizeof(float);
     const size_t tick = (size_t)p->seqs * sizeof(int);
     const size_t freq = (size_t)(c->D / 2) * sizeof(float);
     size_t off = 0;
@@ -107,14 +107,52 @@ struct kivi_cache {
     float *partials;
     int *tickets, *err;
     float *inv_freq;
-    long long n_q;
+    long long n_q;   // the split of every sequence, while the lengths agree
     int r;
     bool prefilled;
+    // Batch elements of different lengths: element b's sequences hold nq_b[b]
+    // quantized and r_b[b] residual tokens (the vectors are valid while
+    // `ragged`; n_q and r otherwise).
+    bool ragged;
+    std::vector<long long> nq_b;
+    std::vector<int> r_b;
     int wg, wr;
     int expire_first_wait;   // testing only (kivi_debug_expire_first_wait)
 };
 
 namespace {
+
+long long nq_at(const kivi_cache *c, int b) { return c->ragged ? c->nq_b[b] : c->n_q; }
+int r_at(const kivi_cache *c, int b) { return c->ragged ? c->r_b[b] : c->r; }
+
+// After per-element updates: if every element holds the same split again,
+// the cache is uniform.
+void settle(kivi_cache *c)
+{
+    bool same = true;
+    for (int b = 1; b < c->cfg.B && same; ++b)
+        same = c->nq_b[b] == c->nq_b[0] && c->r_b[b] == c->r_b[0];
+    c->ragged = !same;
+    if (same) {
+        c->n_q = c->nq_b[0];
+        c->r = c->r_b[0];
+    }
+}
+
+// The decode split of a ragged cache: per batch element its groups, its
+// residual tokens and where its work starts.
+void ragged_table(const kivi_cache *c, RaggedTab *rt)
+{
+    const int B = c->cfg.B, H = c->cfg.H_kv;
+    rt->nb = B;
+    rt->off[0] = 0;
+    for (int b = 0; b < B; ++b) {
+        rt->ng[b] = (int)(c->nq_b[b] / kG);
+        rt->r[b] = c->r_b[b];
+        const long long C = (long long)rt->ng[b] * c->wg + (long long)((rt->r[b] + kResTok - 1) / kResTok) * c->wr;
+        rt->off[b + 1] = rt->off[b] + (long long)H * C;
+    }
+}
 
 // Every call that touches a cache's device memory must run with the cache's
 // device current: its launches, scratch and SM count belong to that device.
@@ -211,6 +249,15 @@ kivi_status kivi_cache_create_ex(const kivi_config *cfg, kivi_cache **out)
     c->n_q = 0;
     c->r = 0;
     c->prefilled = false;
+    c->ragged = false;
+    try {
+        c->nq_b.assign(cfg->B, 0);
+        c->r_b.assign(cfg->B, 0);
+    } catch (...) {
+        if (c->owns) cudaFree(c->base);
+        delete c;
+        return KIVI_ERR_OOM;
+    }
     c->expire_first_wait = 0;
     c->wg = env_int("KIVI_SPLIT_WG", 4);
     c->wr = env_int("KIVI_SPLIT_WR", 3);
@@ -249,14 +296,24 @@ kivi_status kivi_cache_reset(kivi_cache *c)
     c->n_q = 0;
     c->r = 0;
     c->prefilled = false;
+    c->ragged = false;
     return KIVI_OK;
 }
 
 kivi_status kivi_cache_length(const kivi_cache *c, long long *n_q, int *r)
 {
     if (!c || !n_q || !r) return KIVI_ERR_ARG;
+    if (c->ragged) return KIVI_ERR_STATE;
     *n_q = c->n_q;
     *r = c->r;
+    return KIVI_OK;
+}
+
+kivi_status kivi_cache_length_at(const kivi_cache *c, int b, long long *n_q, int *r)
+{
+    if (!c || !n_q || !r || b < 0 || b >= c->cfg.B) return KIVI_ERR_ARG;
+    *n_q = nq_at(c, b);
+    *r = r_at(c, b);
     return KIVI_OK;
 }
 
@@ -296,19 +353,156 @@ kivi_status kivi_prefill(kivi_cache *c, const void *K, const void *V, long long 
     q.r_copy = r;
     q.copy_row0 = n_q;
     q.newK = q.newV = nullptr;
-    cudaError_t e = launch_quant(D, c->cfg.dtype, q, (cudaStream_t)stream);
+    cudaError_t e = launch_quant(D, c->cfg.dtype, q, nullptr, (cudaStream_t)stream);
     if (e != cudaSuccess) return KIVI_ERR_CUDA;
     c->n_q = n_q;
     c->r = r;
+    c->ragged = false;
     c->prefilled = true;
     return KIVI_OK;
 }
+
+kivi_status kivi_prefill_ragged(kivi_cache *c, const void *K, const void *V, long long T_pad,
+                                const long long *T_b, void *stream)
+{
+    if (!c || !K || !V || !T_b || !aligned16(K) || !aligned16(V)) return KIVI_ERR_ARG;
+    if (!on_cache_device(c)) return KIVI_ERR_ARG;
+    if (c->prefilled) return KIVI_ERR_STATE;
+    const int B = c->cfg.B, H = c->cfg.H_kv, R = c->cfg.R, D = c->cfg.D;
+    if (B > kMaxRaggedB) return KIVI_ERR_UNSUPPORTED;
+    if (T_pad < 1) return KIVI_ERR_ARG;
+    if (T_pad > c->cfg.T_max) return KIVI_ERR_CAPACITY;
+    for (int b = 0; b < B; ++b)
+        if (T_b[b] < 1 || T_b[b] > T_pad) return KIVI_ERR_ARG;
+    // One segment per run of consecutive batch elements of one length.
+    QuantSegs sg;
+    sg.nseg = 0;
+    sg.item0[0] = 0;
+    for (int b = 0; b < B; ++b) {
+        const long long n_q = (long long)R * ((T_b[b] - 1) / R);
+        const int r = (int)(T_b[b] - n_q), n_g = (int)(n_q / kG);
+        const int k = sg.nseg - 1;
+        if (k >= 0 && sg.n_g[k] == n_g && sg.r_copy[k] == r) {
+            sg.nseq[k] += H;
+        } else {
+            sg.seq0[sg.nseg] = b * H;
+            sg.nseq[sg.nseg] = H;
+            sg.n_g[sg.nseg] = n_g;
+            sg.g_dst0[sg.nseg] = 0;
+            sg.r_copy[sg.nseg] = r;
+            sg.copy_row0[sg.nseg] = (int)n_q;
+            ++sg.nseg;
+        }
+    }
+    for (int k = 0; k < sg.nseg; ++k)
+        sg.item0[k + 1] = sg.item0[k] + (long long)sg.nseq[k] * (sg.n_g[k] + 1);
+    QuantParams q;
+    q.srcK = (const uint16_t *)K;
+    q.srcV = (const uint16_t *)V;
+    q.src_seq_rows = T_pad;
+    q.packed = c->packed;
+    q.ngcap = c->plan.ngcap;
+    q.g_dst0 = 0;
+    q.n_g = 1;
+    q.seqs = c->plan.seqs;
+    q.resK = c->resK;
+    q.resV = c->resV;
+    q.R = R;
+    q.r_copy = 0;
+    q.copy_row0 = 0;
+    q.newK = q.newV = nullptr;
+    cudaError_t e = launch_quant(D, c->cfg.dtype, q, &sg, (cudaStream_t)stream);
+    if (e != cudaSuccess) return KIVI_ERR_CUDA;
+    for (int b = 0; b < B; ++b) {
+        c->nq_b[b] = (long long)R * ((T_b[b] - 1) / R);
+        c->r_b[b] = (int)(T_b[b] - c->nq_b[b]);
+    }
+    settle(c);
+    c->prefilled = true;
+    return KIVI_OK;
+}
+
+namespace {
+
+// Append to a ragged cache: batch elements whose residual is full flush it
+// (one quantizer launch over segments of them), the others take the token
+// in their own slot.
+kivi_status append_ragged(kivi_cache *c, const void *k_t, const void *v_t, cudaStream_t st)
+{
+    const int B = c->cfg.B, H = c->cfg.H_kv, R = c->cfg.R, D = c->cfg.D;
+    for (int b = 0; b < B; ++b)
+        if (c->nq_b[b] + c->r_b[b] + 1 > c->cfg.T_max) return KIVI_ERR_CAPACITY;
+    QuantSegs sg;
+    sg.nseg = 0;
+    sg.item0[0] = 0;
+    SlotTab sl;
+    bool plain = false;
+    for (int b = 0; b < B; ++b) {
+        if (c->r_b[b] == R) {
+            sl.slot[b] = -1;
+            const int k = sg.nseg - 1;
+            const int g_dst0 = (int)(c->nq_b[b] / kG);
+            if (k >= 0 && sg.seq0[k] + sg.nseq[k] == b * H && sg.g_dst0[k] == g_dst0) {
+                sg.nseq[k] += H;
+            } else {
+                sg.seq0[sg.nseg] = b * H;
+                sg.nseq[sg.nseg] = H;
+                sg.n_g[sg.nseg] = R / kG;
+                sg.g_dst0[sg.nseg] = g_dst0;
+                sg.r_copy[sg.nseg] = 0;
+                sg.copy_row0[sg.nseg] = 0;
+                ++sg.nseg;
+            }
+        } else {
+            sl.slot[b] = c->r_b[b];
+            plain = true;
+        }
+    }
+    for (int k = 0; k < sg.nseg; ++k) sg.item0[k + 1] = sg.item0[k] + (long long)sg.nseq[k] * sg.n_g[k];
+    cudaError_t e = cudaSuccess;
+    if (sg.nseg > 0) {
+        QuantParams q;
+        q.srcK = c->resK;
+        q.srcV = c->resV;
+        q.src_seq_rows = R;
+        q.packed = c->packed;
+        q.ngcap = c->plan.ngcap;
+        q.g_dst0 = 0;
+        q.n_g = R / kG;
+        q.seqs = c->plan.seqs;
+        q.resK = c->resK;
+        q.resV = c->resV;
+        q.R = R;
+        q.r_copy = 0;
+        q.copy_row0 = 0;
+        q.newK = (const uint16_t *)k_t;
+        q.newV = (const uint16_t *)v_t;
+        e = launch_quant(D, c->cfg.dtype, q, &sg, st);
+    }
+    if (e == cudaSuccess && plain)
+        e = launch_append_slots(D, (const uint16_t *)k_t, (const uint16_t *)v_t, c->resK, c->resV,
+                                c->plan.seqs, H, R, sl, st);
+    if (e != cudaSuccess) return KIVI_ERR_CUDA;
+    for (int b = 0; b < B; ++b) {
+        if (c->r_b[b] == R) {
+            c->nq_b[b] += R;
+            c->r_b[b] = 1;
+        } else {
+            c->r_b[b] += 1;
+        }
+    }
+    settle(c);
+    return KIVI_OK;
+}
+
+}  // namespace
 
 kivi_status kivi_append(kivi_cache *c, const void *k_t, const void *v_t, void *stream)
 {
     if (!c || !k_t || !v_t || !aligned16(k_t) || !aligned16(v_t)) return KIVI_ERR_ARG;
     if (!on_cache_device(c)) return KIVI_ERR_ARG;
     if (!c->prefilled) return KIVI_ERR_STATE;
+    if (c->ragged) return append_ragged(c, k_t, v_t, (cudaStream_t)stream);
     if (c->n_q + c->r + 1 > c->cfg.T_max) return KIVI_ERR_CAPACITY;
     const int R = c->cfg.R, D = c->cfg.D;
     cudaError_t e;
@@ -329,7 +523,7 @@ kivi_status kivi_append(kivi_cache *c, const void *k_t, const void *v_t, void *s
         q.copy_row0 = 0;
         q.newK = (const uint16_t *)k_t;
         q.newV = (const uint16_t *)v_t;
-        e = launch_quant(D, c->cfg.dtype, q, (cudaStream_t)stream);
+        e = launch_quant(D, c->cfg.dtype, q, nullptr, (cudaStream_t)stream);
         if (e != cudaSuccess) return KIVI_ERR_CUDA;
         c->n_q += R;
         c->r = 1;
@@ -348,44 +542,61 @@ kivi_status kivi_append_decode(kivi_cache *c, const void *k_t, const void *v_t, 
     if (!c || !k_t || !v_t || !aligned16(k_t) || !aligned16(v_t)) return KIVI_ERR_ARG;
     if (!on_cache_device(c)) return KIVI_ERR_ARG;
     if (!c->prefilled) return KIVI_ERR_STATE;
-    if (c->n_q + c->r + 1 > c->cfg.T_max) return KIVI_ERR_CAPACITY;
-    if (c->r == c->cfg.R) {   // a flush is due: the quantizer runs first
+    bool flush = false;
+    for (int b = 0; b < c->cfg.B; ++b) {
+        if (nq_at(c, b) + r_at(c, b) + 1 > c->cfg.T_max) return KIVI_ERR_CAPACITY;
+        flush = flush || r_at(c, b) == c->cfg.R;
+        if (!c->ragged) break;
+    }
+    if (flush) {   // a flush is due: the quantizer runs first
         const kivi_status st = kivi_append(c, k_t, v_t, stream);
         return st != KIVI_OK ? st : kivi_decode_attn(c, q, H_q, out, stream);
     }
     // The split sees the token already appended; undone if anything fails
     // before the launch.
-    c->r += 1;
+    auto bump = [&](int d) {
+        if (c->ragged)
+            for (int b = 0; b < c->cfg.B; ++b) c->r_b[b] += d;
+        else
+            c->r += d;
+    };
+    bump(1);
     DecodeParams p;
+    RaggedTab rt;
+    bool ragged = false;
+    long long rows = 0;
     int D = 0, HG = 0, dtype = 0, pre_rope = 0;
-    kivi_status st = decode_params_external_scratch(c, q, H_q, out, &p, &D, &HG, &dtype, &pre_rope);
-    if (st == KIVI_OK && p.slots > c->plan.slots) st = KIVI_ERR_UNSUPPORTED;
+    kivi_status st = decode_params_external_scratch(c, q, H_q, out, &p, &D, &HG, &dtype, &pre_rope, &rt,
+                                                    &ragged, &rows);
+    if (st == KIVI_OK && rows > c->plan.part_rows) st = KIVI_ERR_UNSUPPORTED;
     if (st != KIVI_OK) {
-        c->r -= 1;
+        bump(-1);
         return st;
     }
     p.partials = c->partials;
     p.tickets = c->tickets;
-    p.slots = c->plan.slots;
     p.newK = (const uint16_t *)k_t;
     p.newV = (const uint16_t *)v_t;
-    p.new_slot = c->r - 1;
-    const cudaError_t e = launch_decode(D, HG, dtype, pre_rope, p, (cudaStream_t)stream);
-    if (e != cudaSuccess) c->r -= 1;
+    p.new_slot = c->ragged ? -1 : c->r - 1;   // ragged: each sequence's r - 1, in the kernel
+    const cudaError_t e = launch_decode(D, HG, dtype, pre_rope, p, ragged ? &rt : nullptr, (cudaStream_t)stream);
+    if (e != cudaSuccess) bump(-1);
     return cuda_status(e);
 }
 
 kivi_status kivi_decode_attn(kivi_cache *c, const void *q, int H_q, float *out, void *stream)
 {
     DecodeParams p;
+    RaggedTab rt;
+    bool ragged = false;
+    long long rows = 0;
     int D = 0, HG = 0, dtype = 0, pre_rope = 0;
-    kivi_status st = decode_params_external_scratch(c, q, H_q, out, &p, &D, &HG, &dtype, &pre_rope);
+    kivi_status st = decode_params_external_scratch(c, q, H_q, out, &p, &D, &HG, &dtype, &pre_rope, &rt,
+                                                    &ragged, &rows);
     if (st != KIVI_OK) return st;
+    if (rows > c->plan.part_rows) return KIVI_ERR_UNSUPPORTED;
     p.partials = c->partials;
     p.tickets = c->tickets;
-    if (p.slots > c->plan.slots) return KIVI_ERR_UNSUPPORTED;
-    p.slots = c->plan.slots;
-    cudaError_t e = launch_decode(D, HG, dtype, pre_rope, p, (cudaStream_t)stream);
+    cudaError_t e = launch_decode(D, HG, dtype, pre_rope, p, ragged ? &rt : nullptr, (cudaStream_t)stream);
     return cuda_status(e);
 }
 
@@ -484,8 +695,14 @@ extern "C" kivi_status kivi_export(const kivi_cache *c, long long seq0, long lon
     if (!c || seq0 < 0 || nseq < 0 || seq0 + nseq > c->plan.seqs) return KIVI_ERR_ARG;
     if (!c->prefilled) return KIVI_ERR_STATE;
     if (nseq == 0) return KIVI_OK;
-    const int D = c->cfg.D, R = c->cfg.R;
-    const long long n_g = c->n_q / kG;
+    const int D = c->cfg.D, R = c->cfg.R, H = c->cfg.H_kv;
+    // The sequences exported share one split (all of them, unless ragged).
+    const int b0 = (int)(seq0 / H), b1 = (int)((seq0 + nseq - 1) / H);
+    const long long n_q = nq_at(c, b0);
+    const int r = r_at(c, b0);
+    for (int b = b0 + 1; b <= b1; ++b)
+        if (nq_at(c, b) != n_q || r_at(c, b) != r) return KIVI_ERR_ARG;
+    const long long n_g = n_q / kG;
     const size_t gb = (size_t)24 * D;
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return KIVI_ERR_CUDA;
@@ -500,12 +717,12 @@ extern "C" kivi_status kivi_export(const kivi_cache *c, long long seq0, long lon
     const size_t row = (size_t)D * 2;
     const size_t off = (size_t)seq0 * R * D;
     if (resK) {
-        e = cudaMemcpy2D(resK, c->r * row, c->resK + off, (size_t)R * row, c->r * row, nseq,
+        e = cudaMemcpy2D(resK, r * row, c->resK + off, (size_t)R * row, r * row, nseq,
                          cudaMemcpyDeviceToHost);
         if (e != cudaSuccess) return KIVI_ERR_CUDA;
     }
     if (resV) {
-        e = cudaMemcpy2D(resV, c->r * row, c->resV + off, (size_t)R * row, c->r * row, nseq,
+        e = cudaMemcpy2D(resV, r * row, c->resV + off, (size_t)R * row, r * row, nseq,
                          cudaMemcpyDeviceToHost);
         if (e != cudaSuccess) return KIVI_ERR_CUDA;
     }
@@ -538,22 +755,33 @@ namespace kivi {
 // tickets) and the partial slot count left for the caller to fill.
 kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q, float *out,
                                            DecodeParams *p, int *D, int *HG, int *dtype,
-                                           int *pre_rope)
+                                           int *pre_rope, RaggedTab *rt, bool *ragged, long long *rows)
 {
-    if (!c || !q || !out || !p || !aligned16(q) || !aligned16(out)) return KIVI_ERR_ARG;
+    if (!c || !q || !out || !p || !rt || !ragged || !rows || !aligned16(q) || !aligned16(out))
+        return KIVI_ERR_ARG;
     if (!on_cache_device(c)) return KIVI_ERR_ARG;
     if (!c->prefilled) return KIVI_ERR_STATE;
     if (H_q < 1 || H_q % c->cfg.H_kv != 0) return KIVI_ERR_ARG;
     const int hg = H_q / c->cfg.H_kv;
     const int nw = decode_warps_per_cta(c->cfg.D, hg, c->cfg.pre_rope);
     if (nw == 0 || hg > kMaxGroupHeads) return KIVI_ERR_UNSUPPORTED;
+    *ragged = c->ragged;
     Split sp;
-    sp.init(c->plan.seqs, c->n_q / kG, c->r, c->wg, c->wr, 1);
-    long long warps = (long long)c->sms * nw;
-    if (warps > sp.Tot) warps = sp.Tot;
-    sp.init(c->plan.seqs, c->n_q / kG, c->r, c->wg, c->wr, warps);
+    long long Tot, warps = (long long)c->sms * nw;
+    if (c->ragged) {
+        ragged_table(c, rt);
+        Tot = rt->off[rt->nb];
+        if (warps > Tot) warps = Tot;
+        sp.init(c->plan.seqs, rt->ng[0], rt->r[0], c->wg, c->wr, warps);
+        sp.Tot = Tot;
+    } else {
+        sp.init(c->plan.seqs, c->n_q / kG, c->r, c->wg, c->wr, 1);
+        if (warps > sp.Tot) warps = sp.Tot;
+        sp.init(c->plan.seqs, c->n_q / kG, c->r, c->wg, c->wr, warps);
+        Tot = sp.Tot;
+    }
     // The split's divisions are exact for numerators below 2^53 (div_floor).
-    if ((double)sp.Tot * (double)(warps + 1) >= 9007199254740992.0) return KIVI_ERR_UNSUPPORTED;
+    if ((double)Tot * (double)(warps + 1) >= 9007199254740992.0) return KIVI_ERR_UNSUPPORTED;
     sp.set_magics();
     p->div_C = sp.mC;
     p->div_Tot = sp.mT;
@@ -574,13 +802,13 @@ kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q
     p->H_kv = c->cfg.H_kv;
     p->H_q = H_q;
     p->seqs = c->plan.seqs;
-    p->n_groups = c->n_q / kG;
-    p->r = c->r;
-    p->n_q = c->n_q;
+    p->n_groups = c->ragged ? 0 : c->n_q / kG;
+    p->r = c->ragged ? 1 : c->r;
+    p->n_q = c->ragged ? 0 : c->n_q;
     p->wg = c->wg;
     p->wr = c->wr;
     p->warps = warps;
-    p->slots = (int)(warps / p->seqs + 2);
+    *rows = warps + p->seqs;
     p->qscale = (float)(1.4426950408889634 / std::sqrt((double)c->cfg.D));
     p->inv_freq = c->inv_freq;
     p->newK = p->newV = nullptr;

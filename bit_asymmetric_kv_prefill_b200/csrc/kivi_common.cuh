@@ -262,4 +262,19 @@ struct Split {
     }
 };
 
+// ---------------------------------------------------------------------------
+// Per-batch-element lengths of a ragged cache (batch element b's sequences,
+// b*H_kv .. b*H_kv + H_kv - 1, hold n_q = ng[b]*kG quantized and r[b]
+// residual tokens).  The decode split concatenates the sequences' weights
+// (ng*wg + ceil(r/kResTok)*wr each); off[b] is where element b's first
+// sequence starts and off[nb] the total.  Passed to kernels by value.
+// ---------------------------------------------------------------------------
+constexpr int kMaxRaggedB = 512;
+struct RaggedTab {
+    int nb;
+    int ng[kMaxRaggedB];
+    int r[kMaxRaggedB];
+    long long off[kMaxRaggedB + 1];
+};
+
 }  // namespace kivi

@@ -119,9 +119,8 @@ struct DecodeShape {
 };
 
 // ---- the kernel ---------------------------------------------------------------
-template <int D, int HG, int DT, bool ROPE>
-__global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
-    decode_kernel(const DecodeParams p)
+template <int D, int HG, int DT, bool ROPE, bool RAGGED>
+__device__ __forceinline__ void decode_body(const DecodeParams &p, const RaggedTab *rt)
 {
     using L = Layout<D>;
     using W = WarpSmem<D, HG, ROPE>;
@@ -164,19 +163,91 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     sp.mW = p.div_warps;
     sp.mG = p.div_wg;
     sp.mR = p.div_wr;
+    if constexpr (RAGGED) sp.Tot = rt->off[rt->nb];
+    // Per-sequence lengths and work layout: one length for every sequence,
+    // or (ragged caches) the lengths of the sequence's batch element.
+    auto elem = [&](int s) { return (int)div_floor(s, p.div_Hkv); };
+    auto ng_of = [&](int s) -> int {
+        if constexpr (RAGGED) return rt->ng[elem(s)];
+        else return (int)p.n_groups;
+    };
+    auto r_of = [&](int s) -> int {
+        if constexpr (RAGGED) return rt->r[elem(s)];
+        else return p.r;
+    };
+    auto nq_of = [&](int s) -> long long {
+        if constexpr (RAGGED) return (long long)rt->ng[elem(s)] * kG;
+        else return p.n_q;
+    };
+    // The appended token's residual slot (fused append), -1 if none.
+    auto new_slot_of = [&](int s) -> int {
+        if constexpr (RAGGED) return p.newK != nullptr ? r_of(s) - 1 : -1;
+        else return p.new_slot;
+    };
+    auto C_of = [&](int s) -> long long {
+        if constexpr (RAGGED) return (long long)ng_of(s) * p.wg + (long long)((r_of(s) + kResTok - 1) / kResTok) * p.wr;
+        else return sp.C;
+    };
+    auto start_of = [&](int s) -> long long {
+        if constexpr (RAGGED) {
+            const int b = elem(s);
+            return rt->off[b] + (long long)(s - b * p.H_kv) * C_of(s);
+        } else {
+            return (long long)s * sp.C;
+        }
+    };
+    auto seq_of = [&](long long pos) -> int {
+        if constexpr (RAGGED) {
+            int lo_b = 0, hi_b = rt->nb - 1;   // the last element with off[b] <= pos
+            while (lo_b < hi_b) {
+                const int mid = (lo_b + hi_b + 1) >> 1;
+                if (rt->off[mid] <= pos) lo_b = mid;
+                else hi_b = mid - 1;
+            }
+            const int s0 = lo_b * p.H_kv;
+            return s0 + (int)((pos - rt->off[lo_b]) / C_of(s0));
+        } else {
+            return (int)sp.seq_of(pos);
+        }
+    };
+    // Items of sequence s owned by warp w: [first, second).
+    auto items_of = [&](int s, long long w) -> ItemRange {
+        if constexpr (RAGGED) {
+            const long long base = start_of(s), C = C_of(s);
+            const long long ng = ng_of(s), nit = ng + (r_of(s) + kResTok - 1) / kResTok;
+            const long long a = sp.lo(w), b2 = sp.lo(w + 1);
+            const long long ra = a > base ? a - base : 0;
+            const long long rb = b2 < base + C ? b2 - base : C;
+            if (ra >= rb) return ItemRange{0, 0};
+            auto first_at = [&](long long rel) -> long long {
+                const long long gend = ng * p.wg;
+                if (ng > 0 && rel <= gend - p.wg) return div_floor(rel + p.wg - 1, p.div_wg);
+                if (rel <= gend) return ng;
+                const long long idx = ng + div_floor(rel - gend + p.wr - 1, p.div_wr);
+                return idx < nit ? idx : nit;
+            };
+            const long long i0 = first_at(ra), i1 = first_at(rb);
+            return ItemRange{i0, i1 < i0 ? i0 : i1};
+        } else {
+            return sp.items(s, w);
+        }
+    };
+    auto n_items_of = [&](int s) -> int {
+        if constexpr (RAGGED) return ng_of(s) + (r_of(s) + kResTok - 1) / kResTok;
+        else return (int)sp.n_items();
+    };
     // (The warp index enters as an opaque register: measured, this keeps the
     // split's 64-bit arithmetic on the vector pipes and the prologue short.)
     long long gwo = gw;
     asm volatile("" : "+l"(gwo));
     const long long lo = sp.lo(gwo), hi = sp.lo(gwo + 1);
-    const int s_first = (int)sp.seq_of(lo), s_last = (int)sp.seq_of(hi - 1);
-    const int n_items = (int)sp.n_items(), n_groups = (int)p.n_groups;
+    const int s_first = seq_of(lo), s_last = seq_of(hi - 1);
     int i_first, i_end;
-    i_first = (int)sp.items(s_first, gwo).first;
-    i_end = (int)sp.items(s_last, gwo).second;
+    i_first = (int)items_of(s_first, gwo).first;
+    i_end = (int)items_of(s_last, gwo).second;
     auto seq_items = [&](int s, int *i0, int *i1) {
         *i0 = s == s_first ? i_first : 0;
-        *i1 = s == s_last ? i_end : n_items;
+        *i1 = s == s_last ? i_end : n_items_of(s);
         if (*i1 < *i0) *i1 = *i0;
     };
 
@@ -214,15 +285,16 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         const uint32_t bar = bar0 + 8 * ist;
         const uint32_t dst = ring_s + ist * L::GB;
         ist = ist + 1 == kSt ? 0 : ist + 1;
-        if (pf_i < n_groups) {
+        const int pf_ng = ng_of(pf_s);
+        if (pf_i < pf_ng) {
             const uint8_t *src = p.packed + ((long long)pf_s * p.ngcap + pf_i) * (long long)L::GB;
             lane0_expect_copy(lane, bar, dst, src, L::GB, L::GB);
         } else {
-            const int t0 = (pf_i - n_groups) * kResTok;
-            const int nt = min(kResTok, p.r - t0);
+            const int t0 = (pf_i - pf_ng) * kResTok;
+            const int nt = min(kResTok, r_of(pf_s) - t0);
             const uint32_t bytes = (uint32_t)nt * D * 2;
             const long long row = (long long)pf_s * p.R + t0;
-            const int nn = p.new_slot - t0;   // the appended token's row in this slice
+            const int nn = new_slot_of(pf_s) - t0;   // the appended token's row in this slice
             if (p.newK != nullptr && nn >= 0 && nn < nt) {
                 // Fused append: the slice's last row comes from the caller's
                 // k_t/v_t (slot new_slot, the residual's newest); the rows
@@ -288,6 +360,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         int i0, i1;
         seq_items(s, &i0, &i1);
         const int b = (int)div_floor(s, p.div_Hkv), hk = s - b * p.H_kv;
+        const int n_groups = ng_of(s), r_s = r_of(s), new_slot = new_slot_of(s);
+        const long long n_q_s = nq_of(s);
 
         // Scaled query in shared memory (fp32) and the lane's q' inputs; then
         // the next sequence's query is requested (with four or more query
@@ -722,15 +796,15 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
             } else {
                 // ---------------- residual slice of up to 6 tokens ----------------
                 const int t0 = (it - n_groups) * kResTok;
-                const int nt = min(kResTok, p.r - t0);
+                const int nt = min(kResTok, r_s - t0);
                 const uint16_t *rk = (const uint16_t *)st;
                 const uint16_t *rv = (const uint16_t *)(st + kResTok * D * 2);
-                if (p.newK != nullptr && p.new_slot >= t0 && p.new_slot < t0 + nt) {
+                if (p.newK != nullptr && new_slot >= t0 && new_slot < t0 + nt) {
                     // Fused append: this warp persists the new token into its
                     // residual slot (read by later launches' bulk copies).
                     constexpr int C16 = D / 8;   // 16-byte chunks per row
-                    const int nn = p.new_slot - t0;
-                    const long long drow = ((long long)s * p.R + p.new_slot) * D;
+                    const int nn = new_slot - t0;
+                    const long long drow = ((long long)s * p.R + new_slot) * D;
                     for (int c = lane; c < 2 * C16; c += 32) {
                         const int which = c / C16, q16 = c % C16;
                         const uint4 v = *(const uint4 *)((which ? rv : rk) + nn * D + q16 * 8);
@@ -754,7 +828,7 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
                             }
                         }
                         if constexpr (ROPE) {
-                            const float pos = (float)(p.n_q + t0 + tq);
+                            const float pos = (float)(n_q_s + t0 + tq);
 #pragma unroll
                             for (int i = 0; i < HALF; ++i) {
                                 float sn, cn;
@@ -821,8 +895,8 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
         if (failed) break;
 
         // ---------------- this warp's partial for sequence s ----------------
-        const long long first = sp.owner((long long)s * sp.C);
-        const long long last = sp.owner(((long long)s + 1) * sp.C - 1);
+        const long long first = sp.owner(start_of(s));
+        const long long last = sp.owner(start_of(s) + C_of(s) - 1);
         const int count = (int)(last - first + 1);
         const int slot = (int)(gw - first);
         // lt: the softmax sum; zt: the zero term of the lane's value group jl
@@ -868,7 +942,10 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
             }
             continue;
         }
-        float *pbase = p.partials + (((long long)s * p.slots) * HG) * (long long)PSTRIDE;
+        // Compact partial rows: sequence s uses rows first(s) + s + slot, so
+        // the rows of consecutive sequences never meet (first(s + 1) >=
+        // last(s)) and warps + sequences rows serve any split.
+        float *pbase = p.partials + ((first + s) * HG) * (long long)PSTRIDE;
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
             float *prow = pbase + ((long long)slot * HG + h) * PSTRIDE;
@@ -952,6 +1029,21 @@ __global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
     }
 }
 
+template <int D, int HG, int DT, bool ROPE>
+__global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1) decode_kernel(const DecodeParams p)
+{
+    decode_body<D, HG, DT, ROPE, false>(p, nullptr);
+}
+
+// Caches whose batch elements hold different lengths: the same body, lengths
+// per batch element from the table.
+template <int D, int HG, int DT, bool ROPE>
+__global__ void __launch_bounds__(DecodeShape<D, HG, ROPE>::NW * 32, 1)
+    decode_kernel_ragged(const DecodeParams p, const __grid_constant__ RaggedTab rt)
+{
+    decode_body<D, HG, DT, ROPE, true>(p, &rt);
+}
+
 template <int D, int HG, bool ROPE>
 static int warps_per_cta()
 {
@@ -970,31 +1062,39 @@ int decode_warps_per_cta(int D, int HG, int pre_rope)
 }
 
 template <int D, int HG, int DT, bool ROPE>
-static cudaError_t launch_decode_t(const DecodeParams &p, cudaStream_t st)
+static cudaError_t launch_decode_t(const DecodeParams &p, const RaggedTab *rt, cudaStream_t st)
 {
     using S = DecodeShape<D, HG, ROPE>;
-    static PerDeviceOnce once;
-    const cudaError_t e = set_smem_once(once, decode_kernel<D, HG, DT, ROPE>, S::SMEM);
-    if (e != cudaSuccess) return e;
     const long long grid = (p.warps + S::NW - 1) / S::NW;
-    decode_kernel<D, HG, DT, ROPE><<<(unsigned)grid, S::NW * 32, S::SMEM, st>>>(p);
+    if (rt) {
+        static PerDeviceOnce once;
+        const cudaError_t e = set_smem_once(once, decode_kernel_ragged<D, HG, DT, ROPE>, S::SMEM);
+        if (e != cudaSuccess) return e;
+        decode_kernel_ragged<D, HG, DT, ROPE><<<(unsigned)grid, S::NW * 32, S::SMEM, st>>>(p, *rt);
+    } else {
+        static PerDeviceOnce once;
+        const cudaError_t e = set_smem_once(once, decode_kernel<D, HG, DT, ROPE>, S::SMEM);
+        if (e != cudaSuccess) return e;
+        decode_kernel<D, HG, DT, ROPE><<<(unsigned)grid, S::NW * 32, S::SMEM, st>>>(p);
+    }
     return cudaGetLastError();
 }
 
 template <int D, int HG>
-static cudaError_t launch_decode_hg(int dtype, int pre_rope, const DecodeParams &p, cudaStream_t st)
+static cudaError_t launch_decode_hg(int dtype, int pre_rope, const DecodeParams &p, const RaggedTab *rt,
+                                    cudaStream_t st)
 {
     if (dtype) {
-        return pre_rope ? launch_decode_t<D, HG, 1, true>(p, st) : launch_decode_t<D, HG, 1, false>(p, st);
+        return pre_rope ? launch_decode_t<D, HG, 1, true>(p, rt, st) : launch_decode_t<D, HG, 1, false>(p, rt, st);
     }
-    return pre_rope ? launch_decode_t<D, HG, 0, true>(p, st) : launch_decode_t<D, HG, 0, false>(p, st);
+    return pre_rope ? launch_decode_t<D, HG, 0, true>(p, rt, st) : launch_decode_t<D, HG, 0, false>(p, rt, st);
 }
 
 cudaError_t launch_decode(int D, int HG, int dtype, int pre_rope, const DecodeParams &p,
-                          cudaStream_t st)
+                          const RaggedTab *rt, cudaStream_t st)
 {
 #define KIVI_CASE(DD, HH) \
-    if (D == DD && HG == HH) return launch_decode_hg<DD, HH>(dtype, pre_rope, p, st);
+    if (D == DD && HG == HH) return launch_decode_hg<DD, HH>(dtype, pre_rope, p, rt, st);
     KIVI_CASE(64, 1) KIVI_CASE(64, 2) KIVI_CASE(64, 4) KIVI_CASE(64, 8)
     KIVI_CASE(128, 1) KIVI_CASE(128, 2) KIVI_CASE(128, 4) KIVI_CASE(128, 8)
 #undef KIVI_CASE

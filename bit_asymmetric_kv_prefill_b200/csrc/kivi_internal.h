@@ -30,6 +30,25 @@ struct QuantParams {
     Magic div_ng;                 // division by n_g (set by launch_quant)
 };
 
+// Segments of a quantizer launch whose sequences do not share one length
+// (ragged prefill, or a flush of some batch elements): segment k covers
+// sequences [seq0, seq0 + nseq), each quantizing n_g groups from its source
+// rows 0.. into destination groups g_dst0.., then (r_copy > 0) copying source
+// rows [copy_row0, copy_row0 + r_copy) into residual slots 0..  Work items of
+// segment k: [item0[k], item0[k + 1]), the group items first.
+constexpr int kMaxQuantSegs = kMaxRaggedB;
+struct QuantSegs {
+    int nseg;
+    int seq0[kMaxQuantSegs], nseq[kMaxQuantSegs], n_g[kMaxQuantSegs], g_dst0[kMaxQuantSegs];
+    int r_copy[kMaxQuantSegs], copy_row0[kMaxQuantSegs];
+    long long item0[kMaxQuantSegs + 1];
+};
+
+// Residual slot per batch element for an append (-1: the element is skipped).
+struct SlotTab {
+    int slot[kMaxRaggedB];
+};
+
 struct DecodeParams {
     const uint8_t *packed;
     long long ngcap;
@@ -37,7 +56,7 @@ struct DecodeParams {
     int R;
     const uint16_t *q;
     float *out;
-    float *partials;     // [seqs][slots][HG][D+4]
+    float *partials;     // rows of [HG][D+4]: sequence s, partial slot k at row first(s) + s + k
     int *tickets;        // [seqs]
     int *err;            // status word
     int H_kv, H_q;
@@ -48,7 +67,6 @@ struct DecodeParams {
     int wg, wr;          // split weights of a group / a residual item
     long long warps;     // total warps of the split (<= total weight)
     Magic div_C, div_Tot, div_warps, div_wg, div_wr, div_Hkv;   // divisions of the split
-    int slots;           // partial slots per sequence
     float qscale;        // log2(e) / sqrt(D)
     uint32_t magic;      // bits of 2^23 (the code-to-float exponent)
     float neg_magic;     // -2^23
@@ -89,18 +107,28 @@ cudaError_t set_smem_once(PerDeviceOnce &once, Kernel kernel, int bytes)
     return e;
 }
 
-cudaError_t launch_quant(int D, int dtype, const QuantParams &p, cudaStream_t st);
+// segs: null for one length across the sequences (the QuantParams fields),
+// else the segments (QuantParams' n_g, g_dst0, r_copy, copy_row0 unused).
+cudaError_t launch_quant(int D, int dtype, const QuantParams &p, const QuantSegs *segs,
+                         cudaStream_t st);
 cudaError_t launch_append(int D, const uint16_t *k, const uint16_t *v, uint16_t *resK,
                           uint16_t *resV, long long seqs, int R, int slot, cudaStream_t st);
+// Append into per-batch-element slots (slots->slot[b] < 0: element b skipped).
+cudaError_t launch_append_slots(int D, const uint16_t *k, const uint16_t *v, uint16_t *resK,
+                                uint16_t *resV, long long seqs, int H_kv, int R, const SlotTab &slots,
+                                cudaStream_t st);
 // Warps per CTA of the decode kernel for this shape (0 if unsupported).
 int decode_warps_per_cta(int D, int HG, int pre_rope);
+// rt: null for one length across the sequences, else the ragged table.
 cudaError_t launch_decode(int D, int HG, int dtype, int pre_rope, const DecodeParams &p,
-                          cudaStream_t st);
+                          const RaggedTab *rt, cudaStream_t st);
 // Launch parameters of a decode call on cache c, validated as every decode
 // entry point validates them; the scratch pointers (partials, tickets) are
-// left null and `slots` is the least the split needs.
+// left null.  A ragged cache fills *rt and sets *ragged.  *rows is the
+// number of partial rows (each HG x (D + 4) floats) the split needs.
 kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q, float *out,
                                            DecodeParams *p, int *D, int *HG, int *dtype,
-                                           int *pre_rope);
+                                           int *pre_rope, RaggedTab *rt, bool *ragged,
+                                           long long *rows);
 
 }  // namespace kivi

@@ -58,12 +58,15 @@ extern "C" kivi_status kivi_decode_attn_noalloc(kivi_cache *c, const void *q, in
                                                 void *stream)
 {
     kivi::DecodeParams p;
+    kivi::RaggedTab rt;
+    bool ragged = false;
+    long long rows = 0;
     int D = 0, HG = 0, dtype = 0, pre_rope = 0;
     kivi_status st = kivi::decode_params_external_scratch(c, q, H_q, out, &p, &D, &HG, &dtype,
-                                                          &pre_rope);
+                                                          &pre_rope, &rt, &ragged, &rows);
     if (st != KIVI_OK) return st;
     const size_t tick_bytes = ((size_t)p.seqs * sizeof(int) + 255) / 256 * 256;
-    const size_t part_bytes = (size_t)p.seqs * p.slots * HG * (D + 4) * sizeof(float);
+    const size_t part_bytes = (size_t)rows * HG * (D + 4) * sizeof(float);
     if (tick_bytes + part_bytes > kNoAllocScratchBytes) return KIVI_ERR_CAPACITY;
     void *base = nullptr;
     cudaError_t e = scratch_on_current_device(&base);
@@ -75,6 +78,7 @@ extern "C" kivi_status kivi_decode_attn_noalloc(kivi_cache *c, const void *q, in
     p.partials = (float *)((unsigned char *)base + tick_bytes);
     // The array keeps the previous call's contents: the tickets must start at 0.
     e = cudaMemsetAsync(p.tickets, 0, (size_t)p.seqs * sizeof(int), (cudaStream_t)stream);
-    if (e == cudaSuccess) e = kivi::launch_decode(D, HG, dtype, pre_rope, p, (cudaStream_t)stream);
+    if (e == cudaSuccess)
+        e = kivi::launch_decode(D, HG, dtype, pre_rope, p, ragged ? &rt : nullptr, (cudaStream_t)stream);
     return kivi::cuda_status(e);
 }

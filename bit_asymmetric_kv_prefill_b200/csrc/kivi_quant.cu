@@ -201,17 +201,67 @@ struct QuantSmem {
     static constexpr int BYTES = OUTB + 24 * D;
 };
 
+// Work item of a quantizer launch: group g of sequence s (destination group
+// g_dst0 + g), or (copy) the residual copy of sequence s's source rows
+// [copy_row0, copy_row0 + r_copy).
+struct QItem {
+    long long s;
+    int g, g_dst0, r_copy, copy_row0;
+    bool copy;
+};
+
+template <bool SEG>
+__device__ __forceinline__ QItem locate(const QuantParams &p, const QuantSegs *sg, long long item)
+{
+    QItem q;
+    if constexpr (SEG) {
+        int lo = 0, hi = sg->nseg - 1;   // the last segment with item0 <= item
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sg->item0[mid] <= item) lo = mid;
+            else hi = mid - 1;
+        }
+        const long long local = item - sg->item0[lo];
+        const long long ngi = (long long)sg->nseq[lo] * sg->n_g[lo];
+        q.g_dst0 = sg->g_dst0[lo];
+        q.r_copy = sg->r_copy[lo];
+        q.copy_row0 = sg->copy_row0[lo];
+        q.copy = local >= ngi;
+        if (q.copy) {
+            q.s = sg->seq0[lo] + (local - ngi);
+            q.g = 0;
+        } else {
+            const long long si = local / sg->n_g[lo];
+            q.s = sg->seq0[lo] + si;
+            q.g = (int)(local - si * sg->n_g[lo]);
+        }
+    } else {
+        const long long n_group_items = p.seqs * (long long)p.n_g;
+        q.g_dst0 = (int)p.g_dst0;
+        q.r_copy = p.r_copy;
+        q.copy_row0 = (int)p.copy_row0;
+        q.copy = item >= n_group_items;
+        if (q.copy) {
+            q.s = item - n_group_items;
+            q.g = 0;
+        } else {
+            q.s = div_floor(item, p.div_ng);
+            q.g = (int)(item - q.s * p.n_g);
+        }
+    }
+    return q;
+}
+
 template <int D, int DT>
-__device__ void quantize_tile(const QuantParams &p, long long item, const uint16_t *tk,
-                              const uint16_t *tv, uint16_t *thrK, uint16_t *thrV, uint8_t *outb)
+__device__ void quantize_tile(const QuantParams &p, long long s, int g, long long g_dst0,
+                              const uint16_t *tk, const uint16_t *tv, uint16_t *thrK, uint16_t *thrV,
+                              uint8_t *outb)
 {
     using L = Layout<D>;
     using H = In<DT>;
     constexpr int RS = QuantSmem<D>::RS;
     constexpr int NJ = L::NJ, CPL = L::CPL, TPW = L::TPW, KW = L::KW;
     const int tid = threadIdx.x;
-    const long long s = div_floor(item, p.div_ng);
-    const int g = (int)(item - s * p.n_g);
 
     if (tid < D) {
         // Keys, per channel: thread (pair cp, row set hh) takes 16 rows of a
@@ -358,7 +408,7 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
     half_sync<D>(tid);
 
     // Each half stores its own 12*D bytes: [Kc, Km) and [Vc, Vm).
-    uint4 *dst = (uint4 *)(p.packed + ((s * p.ngcap) + p.g_dst0 + g) * (long long)L::GB);
+    uint4 *dst = (uint4 *)(p.packed + ((s * p.ngcap) + g_dst0 + g) * (long long)L::GB);
     {
         const int h = tid < D ? 0 : 1, ht = tid < D ? tid : tid - D;
         const int nthr = tid < D ? D : kQuantThreads - D;
@@ -380,8 +430,8 @@ __device__ void quantize_tile(const QuantParams &p, long long item, const uint16
     }
 }
 
-template <int D, int DT>
-__global__ void __launch_bounds__(kQuantThreads, KIVI_QUANT_CTAS) quant_kernel(QuantParams p)
+template <int D, int DT, bool SEG>
+__device__ __forceinline__ void quant_body(const QuantParams &p, const QuantSegs *sg)
 {
     using S = QuantSmem<D>;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -390,14 +440,17 @@ __global__ void __launch_bounds__(kQuantThreads, KIVI_QUANT_CTAS) quant_kernel(Q
     uint16_t *thrV = (uint16_t *)(smem + S::THRV);
     uint8_t *outb = smem + S::OUTB;
 
-    const long long n_group_items = p.seqs * (long long)p.n_g;
-    const long long n_items = n_group_items + (p.r_copy > 0 ? p.seqs : 0);
+    long long n_items;
+    if constexpr (SEG) n_items = sg->item0[sg->nseg];
+    else n_items = p.seqs * (long long)p.n_g + (p.r_copy > 0 ? p.seqs : 0);
     const int tid = threadIdx.x;
 
     auto issue = [&](long long item, int buf) {
-        if (item >= n_group_items) return;
-        const long long s = div_floor(item, p.div_ng);
-        const int g = (int)(item - s * p.n_g);
+        if (item >= n_items) return;
+        const QItem q = locate<SEG>(p, sg, item);
+        if (q.copy) return;
+        const long long s = q.s;
+        const int g = q.g;
         const long long row0 = s * p.src_seq_rows + (long long)g * 32;
         const uint16_t *k = p.srcK + row0 * D;
         const uint16_t *v = p.srcV + row0 * D;
@@ -421,15 +474,16 @@ __global__ void __launch_bounds__(kQuantThreads, KIVI_QUANT_CTAS) quant_kernel(Q
         cp_async_commit();
         cp_async_wait<1>();
         half_sync<D>(tid);
-        if (item < n_group_items) {
-            quantize_tile<D, DT>(p, item, tiles + (buf * 2 + 0) * S::TILE,
+        const QItem q = locate<SEG>(p, sg, item);
+        if (!q.copy) {
+            quantize_tile<D, DT>(p, q.s, q.g, q.g_dst0, tiles + (buf * 2 + 0) * S::TILE,
                                  tiles + (buf * 2 + 1) * S::TILE, thrK, thrV, outb);
         } else {
             // Prefill residual: rows [copy_row0, copy_row0 + r_copy) -> slots.
-            const long long s = item - n_group_items;
-            const long long n16 = (long long)p.r_copy * (D / 8);
-            const uint4 *sk = (const uint4 *)(p.srcK + (s * p.src_seq_rows + p.copy_row0) * D);
-            const uint4 *sv = (const uint4 *)(p.srcV + (s * p.src_seq_rows + p.copy_row0) * D);
+            const long long s = q.s;
+            const long long n16 = (long long)q.r_copy * (D / 8);
+            const uint4 *sk = (const uint4 *)(p.srcK + (s * p.src_seq_rows + q.copy_row0) * D);
+            const uint4 *sv = (const uint4 *)(p.srcV + (s * p.src_seq_rows + q.copy_row0) * D);
             uint4 *dk = (uint4 *)(p.resK + s * (long long)p.R * D);
             uint4 *dv = (uint4 *)(p.resV + s * (long long)p.R * D);
             const bool kh = tid < D;
@@ -440,6 +494,19 @@ __global__ void __launch_bounds__(kQuantThreads, KIVI_QUANT_CTAS) quant_kernel(Q
         half_sync<D>(tid);
     }
     cp_async_wait<0>();
+}
+
+template <int D, int DT>
+__global__ void __launch_bounds__(kQuantThreads, KIVI_QUANT_CTAS) quant_kernel(QuantParams p)
+{
+    quant_body<D, DT, false>(p, nullptr);
+}
+
+template <int D, int DT>
+__global__ void __launch_bounds__(kQuantThreads, KIVI_QUANT_CTAS)
+    quant_kernel_seg(QuantParams p, const __grid_constant__ QuantSegs sg)
+{
+    quant_body<D, DT, true>(p, &sg);
 }
 
 // Plain append: token rows [seqs][D] -> residual slot `slot` of each sequence.
@@ -457,6 +524,23 @@ __global__ void append_kernel(const uint4 *k, const uint4 *v, uint4 *resK, uint4
     resV[d] = b;
 }
 
+// Append into per-batch-element slots: sequence s = b*H_kv + h takes slot
+// st.slot[b], or nothing when it is negative.
+template <int N16>
+__global__ void append_slots_kernel(const uint4 *k, const uint4 *v, uint4 *resK, uint4 *resV,
+                                    long long seqs, int H_kv, int R, const __grid_constant__ SlotTab st)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= seqs * N16) return;
+    const long long s = i / N16;
+    const int slot = st.slot[s / H_kv];
+    if (slot < 0) return;
+    const long long d = (s * R + slot) * N16 + (i % N16);
+    const uint4 a = __ldcs(k + i), b = __ldcs(v + i);
+    resK[d] = a;
+    resV[d] = b;
+}
+
 int num_sms()
 {
     int dev = 0, n = 0;
@@ -466,26 +550,34 @@ int num_sms()
 }
 
 template <int D, int DT>
-static cudaError_t launch_quant_t(const QuantParams &p, cudaStream_t st)
+static cudaError_t launch_quant_t(const QuantParams &p, const QuantSegs *segs, cudaStream_t st)
 {
     using S = QuantSmem<D>;
-    static PerDeviceOnce once;
-    const cudaError_t e = set_smem_once(once, quant_kernel<D, DT>, S::BYTES);
-    if (e != cudaSuccess) return e;
-    const long long items = p.seqs * (long long)p.n_g + (p.r_copy > 0 ? p.seqs : 0);
+    const long long items = segs ? segs->item0[segs->nseg]
+                                 : p.seqs * (long long)p.n_g + (p.r_copy > 0 ? p.seqs : 0);
     if (items == 0) return cudaSuccess;
     long long grid = (long long)num_sms() * KIVI_QUANT_CTAS;
     if (grid > items) grid = items;
     QuantParams q = p;
     q.div_ng = make_magic((unsigned long long)(p.n_g > 0 ? p.n_g : 1));
-    quant_kernel<D, DT><<<(unsigned)grid, kQuantThreads, S::BYTES, st>>>(q);
+    if (segs) {
+        static PerDeviceOnce once;
+        const cudaError_t e = set_smem_once(once, quant_kernel_seg<D, DT>, S::BYTES);
+        if (e != cudaSuccess) return e;
+        quant_kernel_seg<D, DT><<<(unsigned)grid, kQuantThreads, S::BYTES, st>>>(q, *segs);
+    } else {
+        static PerDeviceOnce once;
+        const cudaError_t e = set_smem_once(once, quant_kernel<D, DT>, S::BYTES);
+        if (e != cudaSuccess) return e;
+        quant_kernel<D, DT><<<(unsigned)grid, kQuantThreads, S::BYTES, st>>>(q);
+    }
     return cudaGetLastError();
 }
 
-cudaError_t launch_quant(int D, int dtype, const QuantParams &p, cudaStream_t st)
+cudaError_t launch_quant(int D, int dtype, const QuantParams &p, const QuantSegs *segs, cudaStream_t st)
 {
-    if (D == 64) return dtype ? launch_quant_t<64, 1>(p, st) : launch_quant_t<64, 0>(p, st);
-    if (D == 128) return dtype ? launch_quant_t<128, 1>(p, st) : launch_quant_t<128, 0>(p, st);
+    if (D == 64) return dtype ? launch_quant_t<64, 1>(p, segs, st) : launch_quant_t<64, 0>(p, segs, st);
+    if (D == 128) return dtype ? launch_quant_t<128, 1>(p, segs, st) : launch_quant_t<128, 0>(p, segs, st);
     return cudaErrorInvalidValue;
 }
 
@@ -501,6 +593,24 @@ cudaError_t launch_append(int D, const uint16_t *k, const uint16_t *v, uint16_t 
     else
         append_kernel<16><<<(unsigned)grid, block, 0, st>>>((const uint4 *)k, (const uint4 *)v,
                                                            (uint4 *)resK, (uint4 *)resV, seqs, R, slot);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_append_slots(int D, const uint16_t *k, const uint16_t *v, uint16_t *resK,
+                                uint16_t *resV, long long seqs, int H_kv, int R, const SlotTab &slots,
+                                cudaStream_t st)
+{
+    const long long total = seqs * (D / 8);
+    const int block = 128;
+    const long long grid = (total + block - 1) / block;
+    if (D == 64)
+        append_slots_kernel<8><<<(unsigned)grid, block, 0, st>>>((const uint4 *)k, (const uint4 *)v,
+                                                                 (uint4 *)resK, (uint4 *)resV, seqs, H_kv, R,
+                                                                 slots);
+    else
+        append_slots_kernel<16><<<(unsigned)grid, block, 0, st>>>((const uint4 *)k, (const uint4 *)v,
+                                                                  (uint4 *)resK, (uint4 *)resV, seqs, H_kv, R,
+                                                                  slots);
     return cudaGetLastError();
 }
 

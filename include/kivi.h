@@ -130,6 +130,25 @@ KIVI_API kivi_status kivi_cache_required_bytes(const kivi_config *cfg, size_t *b
 KIVI_API kivi_status kivi_prefill(kivi_cache *c, const void *K, const void *V, long long T,
                          void *stream);
 
+/*
+ * Prefill a batch whose elements hold different numbers of tokens (the
+ * method's batches are uniform; this serves batches raised to the memory wall
+ * with prompts of mixed lengths, KIVI article paragraph 4).  K, V are
+ * [B, H_kv, T_pad, D] with batch element b's tokens in rows [0, T_b[b]) of
+ * each of its heads; T_b is a HOST array of B lengths, 1 <= T_b[b] <= T_pad
+ * <= T_max.  Each element splits as kivi_prefill would for its own length
+ * (n_q = R*floor((T_b-1)/R) quantized, r = T_b - n_q residual).  Afterwards
+ * kivi_append, kivi_decode_attn, kivi_append_decode and
+ * kivi_decode_attn_noalloc keep their signatures and work per element: an
+ * element whose residual is full flushes on its next append, the others
+ * append in place; decode attends over each element's own tokens.  While the
+ * elements' lengths differ, kivi_cache_length returns KIVI_ERR_STATE (use
+ * kivi_cache_length_at) and kivi_export needs a range of sequences of one
+ * length (e.g. one element's H_kv heads).  B <= 512, else
+ * KIVI_ERR_UNSUPPORTED.  KIVI_ERR_STATE if already prefilled. */
+KIVI_API kivi_status kivi_prefill_ragged(kivi_cache *c, const void *K, const void *V, long long T_pad,
+                                         const long long *T_b, void *stream);
+
 /* Append one token per (batch, kv head).  If the residual holds R tokens they
  * are first quantized as tokens [n_q, n_q+R) (n_q += R, r = 0); the token then
  * goes to residual slot r (r += 1).  KIVI_ERR_CAPACITY past T_max tokens. */
@@ -169,8 +188,9 @@ KIVI_API kivi_status kivi_append_decode(kivi_cache *c, const void *k_t, const vo
  *     whose kernels overlap on the GPU (any caches, any streams) race on the
  *     array: order them, e.g. on one stream.
  *   - Returns KIVI_ERR_CAPACITY, launching nothing, when the call's scratch
- *     (tickets for B*H_kv sequences plus B*H_kv*slots*(H_q/H_kv)*(D+4) fp32
- *     partials, slots = warps/(B*H_kv) + 2) exceeds the array.
+ *     (tickets for B*H_kv sequences plus (warps + B*H_kv) partial rows of
+ *     (H_q/H_kv)*(D+4) fp32, warps being the decode's work streams, at most
+ *     the SM count times 16) exceeds the array.
  * Arguments, layouts and other errors as kivi_decode_attn.
  */
 KIVI_API kivi_status kivi_decode_attn_noalloc(kivi_cache *c, const void *q, int H_q, float *out,
@@ -179,8 +199,12 @@ KIVI_API kivi_status kivi_decode_attn_noalloc(kivi_cache *c, const void *q, int 
 /* Forget the cached tokens (host counters only; device buffers are kept). */
 KIVI_API kivi_status kivi_cache_reset(kivi_cache *c);
 
-/* Current split: n_q quantized tokens, r residual tokens. */
+/* Current split: n_q quantized tokens, r residual tokens (KIVI_ERR_STATE
+ * while the batch elements' lengths differ). */
 KIVI_API kivi_status kivi_cache_length(const kivi_cache *c, long long *n_q, int *r);
+
+/* Current split of batch element b (0 <= b < B). */
+KIVI_API kivi_status kivi_cache_length_at(const kivi_cache *c, int b, long long *n_q, int *r);
 
 /* Allocated device bytes of the cache, by purpose. */
 KIVI_API kivi_status kivi_cache_bytes(const kivi_cache *c, kivi_bytes *out);
