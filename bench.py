@@ -632,6 +632,47 @@ def summarize(wb, t, steps, world, peak):
     }
 
 
+def graph_decode(wb, steps, warmup):
+    """One decode per layer cache (the caches as the last step left them),
+    captured once into a CUDA graph and replayed: the launch overhead of the
+    whole stack amortised.  Device time per replay (CUDA events)."""
+    import torch
+    w, L = wb.w, wb.L
+    qp = [row[l % wb.sets][2] for row in wb.Sp[:1] for l in range(wb.nl)]
+    s = torch.cuda.Stream(wb.dev)
+    s.wait_stream(wb.stream)
+    sp = ctypes.c_void_p(s.cuda_stream)
+
+    def run():
+        bad = 0
+        for l in range(wb.nl):
+            bad |= L.kivi_decode_attn(wb.H[l], qp[l], w.H_q, wb.Op[l], sp)
+        if bad:
+            raise RuntimeError("a KIVI call failed during graph capture")
+
+    with torch.cuda.stream(s):
+        run()
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize(wb.dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize(wb.dev)
+    ms = a.elapsed_time(b) / steps
+    n_q, r, _ = wb.calls[0]
+    per = decode_bytes(w, n_q, r)
+    del g
+    return {"layers": wb.nl, "us_per_replay": 1e3 * ms, "us_per_layer": 1e3 * ms / wb.nl,
+            "achieved_gbs": per * wb.nl / (ms / 1e3) / 1e9, "launches_per_replay": wb.nl}
+
+
 def per_config_entry(args, name, dev, peak):
     """Measure one of the other workloads at full size (rank 0, N = 1)."""
     import torch
@@ -646,6 +687,7 @@ def per_config_entry(args, name, dev, peak):
         tr = traffic_per_launch(w, True)
         s["decode"]["traffic"] = tr
         if name == "llama2_13b_cache":
+            s["decode_graph"] = graph_decode(wb, args.steps, args.warmup)
             nb = wb.caches[0].nbytes()
             per_tok = lambda x: x * layers / (w.B * w.T)
             rec, meta = cache_record_bytes(w, layers)

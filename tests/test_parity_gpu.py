@@ -367,6 +367,42 @@ def test_an_expired_wait_is_reported_and_the_next_call_is_clean(name, kw, fused)
     assert c.device_status() == 0 and a.device_status() == 0
 
 
+def test_decode_of_many_layers_replays_from_a_cuda_graph():
+    """The decode calls allocate nothing and never synchronise, and their
+    lengths travel in the launch parameters: the decodes of a stack of layer
+    caches captured once into a CUDA graph replay to the eager outputs bit
+    for bit, as often as replayed (the merge tickets reset themselves)."""
+    w = small("llama2_13b_cache", B=2, H_q=8, H_kv=4, T=700, layers=1)
+    layers = 6
+    caches, qs = [], []
+    for l in range(layers):
+        K, V = synth.prefill_inputs(w, 30 + l, device=DEV)
+        c = KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, w.T)
+        c.prefill(K, V)
+        caches.append(c)
+        qs.append(synth.step_inputs(w, 0, 30 + l, device=DEV)[2])
+    eager = [c.decode(q) for c, q in zip(caches, qs)]
+    outs = [torch.empty_like(o) for o in eager]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):           # warm-up on the capture stream
+        for c, q, o in zip(caches, qs, outs):
+            c.decode(q, out=o, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for c, q, o in zip(caches, qs, outs):
+            c.decode(q, out=o)
+    for _ in range(3):
+        for o in outs:
+            o.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        for o, e in zip(outs, eager):
+            assert torch.equal(o, e)
+    assert all(c.device_status() == 0 for c in caches)
+
+
 def test_caller_workspace_holds_the_whole_cache():
     w = small("tiny", T=300, B=2, steps=0)
     n = KiviCache.required_bytes(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, 300)
