@@ -772,9 +772,14 @@ def run_e2e(args, wb, world):
     import torch
     w, dev, nl, caches = wb.w, wb.dev, wb.nl, wb.caches
     Ks, Vs, steps = wb.Ks, wb.Vs, [[row[l] for l in range(nl)] for row in wb.steps]
-    hK = [k.cpu().pin_memory() for k in Ks]
-    hV = [v.cpu().pin_memory() for v in Vs]
-    hS = [[tuple(t.cpu().pin_memory() for t in st) for st in row] for row in steps]
+    def pinned(t):   # a pinned host copy, with no pageable copy in between
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    hK = [pinned(k) for k in Ks]
+    hV = [pinned(v) for v in Vs]
+    hS = [[tuple(pinned(t) for t in st) for st in row] for row in steps]
     dK = [torch.empty_like(Ks[0]) for _ in range(nl)]
     dV = [torch.empty_like(Vs[0]) for _ in range(nl)]
     dS = [[[tuple(torch.empty_like(t) for t in steps[0][0]) for _ in range(nl)] for _ in hS]
