@@ -501,10 +501,12 @@ class Workbench:
         self.n_dec = layers * len(self.calls)
         self.launches_step = layers * (1 + len(self.calls) + sum(k == "flush" for _, _, k in self.calls))
 
-    def step(self, dec_ev=None, pre_ev=None):
+    def step(self, runs=None, pre_ev=None, pool=None):
         """One step: every layer's reset and prefill, then the decode calls.
-        Events (CUDA, on the launching stream) bracket each decode launch and
-        each prefill when given."""
+        When timing, events (CUDA, on the launching stream) bracket each
+        prefill and each run of back-to-back decode launches (a flush's
+        quantizer launch ends a run): `runs` receives (start, end, launches)
+        per run, events drawn from `pool`."""
         L, H, sp, w = self.L, self.H, self.sp, self.w
         bad = 0
         for l in range(self.nl):
@@ -515,33 +517,52 @@ class Workbench:
             bad |= L.kivi_prefill(H[l], self.Kp[i], self.Vp[i], w.T, sp)
             if pre_ev is not None:
                 pre_ev[l][1].record(self.stream)
-        j = 0
+        run = None   # [start event, launches] of the open run
+
+        def close_run():
+            nonlocal run
+            if run is not None:
+                e = pool.pop()
+                e.record(self.stream)
+                runs.append((run[0], e, run[1]))
+                run = None
+
         for c, (_, _, kind) in enumerate(self.calls):
             row = self.Sp[c]
             for l in range(self.nl):
                 k, v, q = row[l % self.sets]
                 if kind == "flush":
+                    if runs is not None:
+                        close_run()
                     bad |= L.kivi_append(H[l], k, v, sp)
-                if dec_ev is not None:
-                    dec_ev[j][0].record(self.stream)
+                if runs is not None and run is None:
+                    e = pool.pop()
+                    e.record(self.stream)
+                    run = [e, 0]
                 if kind == "fused":
                     bad |= L.kivi_append_decode(H[l], k, v, q, w.H_q, self.Op[l], sp)
                 else:
                     bad |= L.kivi_decode_attn(H[l], q, w.H_q, self.Op[l], sp)
-                if dec_ev is not None:
-                    dec_ev[j][1].record(self.stream)
-                j += 1
+                if runs is not None:
+                    run[1] += 1
+        if runs is not None:
+            close_run()
         if bad:
             raise RuntimeError("a KIVI call failed during the benchmark")
 
     def measure(self, steps, warmup, clocks=True):
-        """Warm up, then time `steps` steps (device time of the whole region,
-        and of every decode launch and prefill).  Returns a dict of timings."""
+        """Warm up, then time `steps` steps: device time of the whole region,
+        of every prefill, and of every run of back-to-back decode launches
+        (per-launch duration = the runs' total over their launches; an event
+        between every two launches would add its own gap to each).  Returns
+        a dict of timings."""
         import torch
         for _ in range(warmup):
             self.step()
         ev = lambda: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-        dec_ev = [[ev() for _ in range(self.n_dec)] for _ in range(steps)]
+        flush_launches = self.nl * sum(k == "flush" for _, _, k in self.calls)
+        pool = [torch.cuda.Event(enable_timing=True) for _ in range(steps * 2 * (flush_launches + 2))]
+        runs = []
         pre_ev = [[ev() for _ in range(self.nl)] for _ in range(steps)]
         t0e, t1e = ev()
         ck = clock_sampler(self.dev) if clocks else None
@@ -551,7 +572,7 @@ class Workbench:
             time.sleep(0.3)  # let the sampler attach before the timed region
         t0e.record(self.stream)
         for k in range(steps):
-            self.step(dec_ev[k], pre_ev[k])
+            self.step(runs, pre_ev[k], pool)
         t1e.record(self.stream)
         torch.cuda.synchronize(self.dev)
         cks = ck.stop() if ck else None
@@ -559,9 +580,9 @@ class Workbench:
         status = max(c.device_status() for c in self.caches)
         if status != 0:
             raise RuntimeError(f"device status {status} after the timed region")
-        dec_ms = [a.elapsed_time(b) for row in dec_ev for a, b in row]
+        run_ms = [(a.elapsed_time(b), n) for a, b, n in runs]
         pre_ms = [a.elapsed_time(b) for row in pre_ev for a, b in row]
-        return {"ms": t0e.elapsed_time(t1e), "dec_ms": dec_ms, "pre_ms": pre_ms, "clocks": cks}
+        return {"ms": t0e.elapsed_time(t1e), "runs": run_ms, "pre_ms": pre_ms, "clocks": cks}
 
     def close(self):
         for c in self.caches:
@@ -604,7 +625,9 @@ def roofline(wb, dec_avg_ms, t, peak, peak_kind, traffic):
 def summarize(wb, t, steps, world, peak):
     """Per-workload figures from a Workbench measurement."""
     w = wb.w
-    dec_avg = sum(t["dec_ms"]) / len(t["dec_ms"])
+    launches = sum(n for _, n in t["runs"])
+    dec_total = sum(ms for ms, _ in t["runs"])
+    dec_avg = dec_total / launches
     pre_avg = sum(t["pre_ms"]) / len(t["pre_ms"])
     bpl = wb.bytes_step / wb.n_dec
     achieved = bpl / (dec_avg / 1e3) / 1e9
@@ -615,15 +638,16 @@ def summarize(wb, t, steps, world, peak):
     return {
         "value": world * wb.units_step * steps / (t["ms"] / 1e3), "unit": UNIT,
         "ms_per_step": t["ms"] / steps, "steps": steps,
-        "decode": {"avg_us": 1e3 * dec_avg, "median_us": 1e3 * statistics.median(t["dec_ms"]),
-                   "p90_us": 1e3 * sorted(t["dec_ms"])[int(0.9 * (len(t["dec_ms"]) - 1))],
-                   "launches_timed": len(t["dec_ms"]), "alg_bytes_per_launch": bpl,
+        "decode": {"avg_us": 1e3 * dec_avg,
+                   "timing": "CUDA events around each run of back-to-back decode launches",
+                   "runs_timed": len(t["runs"]), "launches_timed": launches,
+                   "alg_bytes_per_launch": bpl,
                    "achieved_gbs": achieved, "frac_of_measured_hbm": achieved / peak,
                    "frac_of_8TBps": achieved / 8000.0,
                    "alg_flops_per_launch": fpl, "achieved_tflops": tfs,
                    "frac_of_fma_peak": tfs / fpk,
                    "tokens_heads_per_s": wb.units_step / wb.n_dec / (dec_avg / 1e3),
-                   "gpu_time_share": sum(t["dec_ms"]) / t["ms"]},
+                   "gpu_time_share": dec_total / t["ms"]},
         "prefill": {"avg_us": 1e3 * pre_avg, "alg_bytes": pb,
                     "achieved_gbs": pb / (pre_avg / 1e3) / 1e9,
                     "frac_of_measured_hbm": pb / (pre_avg / 1e3) / 1e9 / peak,
@@ -725,7 +749,7 @@ def run_gpu(args):
     wb = Workbench(w, layers, sets, rank, dev)
     t = wb.measure(args.steps, args.warmup)
     ms = reduce_max(t["ms"], dev)
-    dec_avg = reduce_max(sum(t["dec_ms"]) / len(t["dec_ms"]), dev)
+    dec_avg = reduce_max(sum(ms_ for ms_, _ in t["runs"]) / sum(n for _, n in t["runs"]), dev)
     t["ms"] = ms
     s = summarize(wb, t, args.steps, world, peak)
     roof = roofline(wb, dec_avg, t, peak, peak_kind,
