@@ -36,6 +36,8 @@
 //    reduction and the hardware sine/cosine.
 //  * With kivi_append_decode the residual slice that holds the appended
 //    token takes it from the caller's k_t/v_t and stores it to the residual.
+#include <utility>
+
 #include <cuda_runtime.h>
 
 #include "kivi_common.cuh"
@@ -56,6 +58,9 @@ namespace kivi {
 #endif
 #ifndef KIVI_DECODE_MAXW_GQA_ROPE
 #define KIVI_DECODE_MAXW_GQA_ROPE 8   // the same with pre-RoPE keys
+#endif
+#ifndef KIVI_PDL
+#define KIVI_PDL 1   // programmatic dependent launch of the decode
 #endif
 #ifndef KIVI_KEYS_SCALAR
 #define KIVI_KEYS_SCALAR 1   // four query heads: key dot products as scalar FMAs
@@ -133,6 +138,11 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const RaggedT
     extern __shared__ __align__(128) unsigned char smem_all[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long gw = (long long)blockIdx.x * NW + warp;
+#if KIVI_PDL
+    // The next launch on the stream may be scheduled as soon as every CTA of
+    // this one has started (it waits for this launch's memory itself).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
     if (gw >= p.warps) return;  // warp-uniform
 
     unsigned char *ws = smem_all + warp * W::BYTES;
@@ -261,6 +271,13 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const RaggedT
 #pragma unroll
         for (int i = 0; i < QW; ++i) qnext[i] = __ldg(qg + lane + 32 * i);
     };
+#if KIVI_PDL
+    // Launched as a programmatic dependent of the previous launch on the
+    // stream: everything above ran while that launch was finishing; from
+    // here on the kernel reads global memory it may have written (the query,
+    // the cache), so it waits for its completion and memory first.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
     load_q(s_first);   // ahead of the ring's copies, which it would queue behind
     __syncwarp();
 
@@ -1061,22 +1078,43 @@ int decode_warps_per_cta(int D, int HG, int pre_rope)
     return 0;
 }
 
+// Launch a decode kernel; with KIVI_PDL as a programmatic dependent of the
+// previous launch on the stream (its CTAs may start while that launch
+// finishes and wait in the kernel before their first global read).
+template <typename... Params, typename... Args>
+static cudaError_t launch_kernel(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
+                                 cudaStream_t st, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = KIVI_PDL ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int D, int HG, int DT, bool ROPE>
 static cudaError_t launch_decode_t(const DecodeParams &p, const RaggedTab *rt, cudaStream_t st)
 {
     using S = DecodeShape<D, HG, ROPE>;
-    const long long grid = (p.warps + S::NW - 1) / S::NW;
+    const unsigned grid = (unsigned)((p.warps + S::NW - 1) / S::NW);
+    cudaError_t e;
     if (rt) {
         static PerDeviceOnce once;
-        const cudaError_t e = set_smem_once(once, decode_kernel_ragged<D, HG, DT, ROPE>, S::SMEM);
-        if (e != cudaSuccess) return e;
-        decode_kernel_ragged<D, HG, DT, ROPE><<<(unsigned)grid, S::NW * 32, S::SMEM, st>>>(p, *rt);
+        e = set_smem_once(once, decode_kernel_ragged<D, HG, DT, ROPE>, S::SMEM);
+        if (e == cudaSuccess)
+            e = launch_kernel(decode_kernel_ragged<D, HG, DT, ROPE>, grid, S::NW * 32, S::SMEM, st, p, *rt);
     } else {
         static PerDeviceOnce once;
-        const cudaError_t e = set_smem_once(once, decode_kernel<D, HG, DT, ROPE>, S::SMEM);
-        if (e != cudaSuccess) return e;
-        decode_kernel<D, HG, DT, ROPE><<<(unsigned)grid, S::NW * 32, S::SMEM, st>>>(p);
+        e = set_smem_once(once, decode_kernel<D, HG, DT, ROPE>, S::SMEM);
+        if (e == cudaSuccess) e = launch_kernel(decode_kernel<D, HG, DT, ROPE>, grid, S::NW * 32, S::SMEM, st, p);
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
