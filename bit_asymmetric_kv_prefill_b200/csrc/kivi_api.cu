@@ -763,7 +763,7 @@ kivi_status decode_params_external_scratch(kivi_cache *c, const void *q, int H_q
     if (!c->prefilled) return KIVI_ERR_STATE;
     if (H_q < 1 || H_q % c->cfg.H_kv != 0) return KIVI_ERR_ARG;
     const int hg = H_q / c->cfg.H_kv;
-    const int nw = decode_warps_per_cta(c->cfg.D, hg, c->cfg.pre_rope);
+    const int nw = decode_warps_per_sm(c->cfg.D, hg, c->cfg.pre_rope);
     if (nw == 0 || hg > kMaxGroupHeads) return KIVI_ERR_UNSUPPORTED;
     *ragged = c->ragged;
     Split sp;

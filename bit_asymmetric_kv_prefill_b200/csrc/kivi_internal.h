@@ -117,8 +117,8 @@ cudaError_t launch_append(int D, const uint16_t *k, const uint16_t *v, uint16_t 
 cudaError_t launch_append_slots(int D, const uint16_t *k, const uint16_t *v, uint16_t *resK,
                                 uint16_t *resV, long long seqs, int H_kv, int R, const SlotTab &slots,
                                 cudaStream_t st);
-// Warps per CTA of the decode kernel for this shape (0 if unsupported).
-int decode_warps_per_cta(int D, int HG, int pre_rope);
+// Resident decode warps per SM for this shape (0 if unsupported).
+int decode_warps_per_sm(int D, int HG, int pre_rope);
 // rt: null for one length across the sequences, else the ragged table.
 cudaError_t launch_decode(int D, int HG, int dtype, int pre_rope, const DecodeParams &p,
                           const RaggedTab *rt, cudaStream_t st);
