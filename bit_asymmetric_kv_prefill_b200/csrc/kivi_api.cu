@@ -27,6 +27,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Plan {
     long long seqs, ngcap;
     long long part_rows;   // decode partial rows: every split has at most warps + seqs
+    long long tick_count;  // decode tickets: one per sequence, one per partial row
     size_t off_packed, off_resK, off_resV, off_part, off_tick, off_err, off_freq, total;
     size_t codes, meta, residual, scratch;
 };
@@ -55,7 +56,8 @@ kivi_status make_plan(const kivi_config *c, int sms, Plan *p)
     const size_t packed = (size_t)p->seqs * p->ngcap * gb;
     const size_t res = (size_t)p->seqs * c->R * c->D * 2;
     const size_t part = (size_t)p->part_rows * kMaxGroupHeads * (c->D + 4) * sizeof(float);
-    const size_t tick = (size_t)p->seqs * sizeof(int);
+    p->tick_count = p->seqs + p->part_rows;
+    const size_t tick = (size_t)p->tick_count * sizeof(int);
     const size_t freq = (size_t)(c->D / 2) * sizeof(float);
     size_t off = 0;
     p->off_packed = off;
@@ -231,7 +233,7 @@ kivi_status kivi_cache_create_ex(const kivi_config *cfg, kivi_cache **out)
     c->tickets = (int *)(c->base + c->plan.off_tick);
     c->err = (int *)(c->base + c->plan.off_err);
     c->inv_freq = (float *)(c->base + c->plan.off_freq);
-    cudaError_t e = cudaMemset(c->tickets, 0, c->plan.seqs * sizeof(int));
+    cudaError_t e = cudaMemset(c->tickets, 0, c->plan.tick_count * sizeof(int));
     if (e == cudaSuccess) e = cudaMemset(c->err, 0, sizeof(int));
     if (e == cudaSuccess && cfg->pre_rope) {
         // inv_freq_i = fp32(theta^(-2i/D)), rounded once from double.
@@ -615,7 +617,7 @@ kivi_status kivi_device_status(kivi_cache *c, int *code)
     if (e == cudaSuccess) e = cudaMemcpy(code, c->err, sizeof(int), cudaMemcpyDeviceToHost);
     if (e == cudaSuccess && *code != 0) {
         e = cudaMemset(c->err, 0, sizeof(int));
-        if (e == cudaSuccess) e = cudaMemset(c->tickets, 0, c->plan.seqs * sizeof(int));
+        if (e == cudaSuccess) e = cudaMemset(c->tickets, 0, c->plan.tick_count * sizeof(int));
         if (e == cudaSuccess) e = cudaDeviceSynchronize();
     }
     return cuda_status(e);

@@ -68,6 +68,9 @@ namespace kivi {
 #ifndef KIVI_KEYS_SCALAR
 #define KIVI_KEYS_SCALAR 1   // four query heads: key dot products as scalar FMAs
 #endif
+#ifndef KIVI_MERGE_FANIN
+#define KIVI_MERGE_FANIN 8   // partials merged per first-level block (0: one level)
+#endif
 #ifndef KIVI_ROPE_UNROLL
 #define KIVI_ROPE_UNROLL 1   // pre-RoPE key loop: pair-steps unrolled (measured best)
 #endif
@@ -385,6 +388,68 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const RaggedT
         for (int e = lane; e < D / 2; e += 32) frq[(e / HALF) * W::FRS + e % HALF] = __ldg(p.inv_freq + e);
         __syncwarp();
     }
+
+    // Log-sum-exp merge of n partial rows of head h: slots k_first,
+    // k_first + k_step, ... of the rows at pbase.  Each round trip loads the
+    // (m, l) and the lane's QPL channels of 8 rows together and folds them
+    // into a running (max, sum, row).  With `dst` the normalised result goes
+    // there; without, the unnormalised merge (a partial of the same form)
+    // replaces row k_first.
+    auto merge_rows = [&](float *pbase, int k_first, int k_step, int n, int h, float *dst) {
+        float M = -INFINITY, lacc = 0.f;
+        float oo[QPL];
+#pragma unroll
+        for (int c = 0; c < QPL; ++c) oo[c] = 0.f;
+        for (int k0 = 0; k0 < n; k0 += 8) {
+            float2 ml[8];
+            float v[8][QPL];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (k0 + j < n) {
+                    const float *row = pbase + ((long long)(k_first + (k0 + j) * k_step) * HG + h) * PSTRIDE;
+                    ml[j] = __ldcg((const float2 *)(row + D));
+#pragma unroll
+                    for (int c = 0; c < QPL; c += 2) {
+                        const float2 x = __ldcg((const float2 *)(row + lane * QPL + c));
+                        v[j][c] = x.x;
+                        v[j][c + 1] = x.y;
+                    }
+                } else {
+                    ml[j] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+                    for (int c = 0; c < QPL; ++c) v[j][c] = 0.f;
+                }
+            }
+            float mx = M;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx = fmaxf(mx, ml[j].x);
+            if (mx == -INFINITY) continue;   // only empty partials so far
+            const float a = ex2(M - mx);
+            lacc *= a;
+#pragma unroll
+            for (int c = 0; c < QPL; ++c) oo[c] *= a;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float wj = ex2(ml[j].x - mx);
+                lacc = fmaf(wj, ml[j].y, lacc);
+#pragma unroll
+                for (int c = 0; c < QPL; ++c) oo[c] = fmaf(wj, v[j][c], oo[c]);
+            }
+            M = mx;
+        }
+        if (dst) {
+            const float inv = 1.0f / lacc;
+#pragma unroll
+            for (int c = 0; c < QPL; c += 2)
+                *(float2 *)(dst + lane * QPL + c) = make_float2(oo[c] * inv, oo[c + 1] * inv);
+        } else {
+            float *row = pbase + ((long long)k_first * HG + h) * PSTRIDE;
+            __syncwarp();   // every lane has read the row's (m, l)
+#pragma unroll
+            for (int c = 0; c < QPL; c += 2) __stcg((float2 *)(row + lane * QPL + c), make_float2(oo[c], oo[c + 1]));
+            if (lane == 0) __stcg((float2 *)(row + D), make_float2(M, lacc));
+        }
+    };
 
     for (int s = s_first; s <= s_last && !failed; ++s) {
         int i0, i1;
@@ -986,67 +1051,47 @@ __device__ __forceinline__ void decode_body(const DecodeParams &p, const RaggedT
             }
             if (lane == 0) *(float2 *)(prow + D) = make_float2(m[h], lt[h]);
         }
+        // Merge.  A sequence split over at most 2F warps is merged by the
+        // last of them in one pass.  Longer ones merge in two levels, so
+        // that no single warp walks every partial at the end: slots are cut
+        // into blocks of F, the last warp of each block folds its block into
+        // the block's first row, and the last block to finish folds those
+        // rows into the output.  Each merge reads its rows in slot order, so
+        // the result does not depend on which warp finishes last.
+        constexpr int F = KIVI_MERGE_FANIN > 0 ? KIVI_MERGE_FANIN : 1;
+        const bool two_level = KIVI_MERGE_FANIN > 0 && count > 2 * F;
+        const int n_blocks = two_level ? (count + F - 1) / F : count;
+        const int kstep = two_level ? F : 1;
+        // Level 0 is this warp's block (only when it holds more than one
+        // partial), level 1 the whole sequence; a warp that is not the last
+        // to arrive at a level leaves the sequence.  (One loop, so that the
+        // merge is generated once.)
+        int kb = 0, k0 = 0, cnt = 0, lvl = 1;
+        if (two_level) {
+            kb = slot / F;
+            k0 = kb * F;
+            cnt = count - k0 < F ? count - k0 : F;
+            if (cnt > 1) lvl = 0;
+        }
         __syncwarp();
-        int is_last = 0;
-        if (lane == 0) {
-            __threadfence();
-            is_last = atomicAdd(p.tickets + s, 1) == count - 1;
-        }
-        is_last = __shfl_sync(FULL, is_last, 0);
-        if (!is_last) continue;
-        __threadfence();
-        // Log-sum-exp merge of the `count` partials of sequence s in one pass:
-        // each round trip loads (m, l) and the lane's channels of 8 partials
-        // together and folds them into a running (max, sum, row).
 #pragma unroll 1
-        for (int h = 0; h < HG; ++h) {
-            float M = -INFINITY, lacc = 0.f;
-            float oo[QPL];
-#pragma unroll
-            for (int c = 0; c < QPL; ++c) oo[c] = 0.f;
-            for (int k0 = 0; k0 < count; k0 += 8) {
-                float2 ml[8];
-                float v[8][QPL];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (k0 + j < count) {
-                        const float *row = pbase + ((long long)(k0 + j) * HG + h) * PSTRIDE;
-                        ml[j] = __ldcg((const float2 *)(row + D));
-#pragma unroll
-                        for (int c = 0; c < QPL; c += 2) {
-                            const float2 x = __ldcg((const float2 *)(row + lane * QPL + c));
-                            v[j][c] = x.x;
-                            v[j][c + 1] = x.y;
-                        }
-                    } else {
-                        ml[j] = make_float2(-INFINITY, 0.f);
-#pragma unroll
-                        for (int c = 0; c < QPL; ++c) v[j][c] = 0.f;
-                    }
-                }
-                float mx = M;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) mx = fmaxf(mx, ml[j].x);
-                if (mx == -INFINITY) continue;   // only empty partials so far
-                const float a = ex2(M - mx);
-                lacc *= a;
-#pragma unroll
-                for (int c = 0; c < QPL; ++c) oo[c] *= a;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float wj = ex2(ml[j].x - mx);
-                    lacc = fmaf(wj, ml[j].y, lacc);
-#pragma unroll
-                    for (int c = 0; c < QPL; ++c) oo[c] = fmaf(wj, v[j][c], oo[c]);
-                }
-                M = mx;
-            }
-            const float inv = 1.0f / lacc;
-#pragma unroll
-            for (int c = 0; c < QPL; c += 2)
-                *(float2 *)(outrow + h * D + lane * QPL + c) = make_float2(oo[c] * inv, oo[c + 1] * inv);
+        for (; lvl < 2; ++lvl) {
+            int *tk = lvl == 0 ? p.tickets + p.seqs + (first + s + kb) : p.tickets + s;
+            const int need = lvl == 0 ? cnt : n_blocks;
+            // Every lane fences its own row stores (one warp instruction
+            // either way) before lane 0 takes the ticket.
+            __threadfence();
+            int last = 0;
+            if (lane == 0) last = atomicAdd(tk, 1) == need - 1;
+            if (!__shfl_sync(FULL, last, 0)) break;
+            __threadfence();
+#pragma unroll 1
+            for (int h = 0; h < HG; ++h)
+                merge_rows(pbase, lvl == 0 ? k0 : 0, lvl == 0 ? 1 : kstep, need, h,
+                           lvl == 0 ? nullptr : outrow + h * D);
+            __syncwarp();
+            if (lane == 0) *tk = 0;
         }
-        if (lane == 0) p.tickets[s] = 0;
     }
 
     if (failed) {

@@ -57,7 +57,7 @@ struct DecodeParams {
     const uint16_t *q;
     float *out;
     float *partials;     // rows of [HG][D+4]: sequence s, partial slot k at row first(s) + s + k
-    int *tickets;        // [seqs]
+    int *tickets;        // [seqs + partial rows]: sequence s at s, merge block of row r at seqs + r
     int *err;            // status word
     int H_kv, H_q;
     long long seqs;

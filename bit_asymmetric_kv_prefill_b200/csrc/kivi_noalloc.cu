@@ -65,7 +65,9 @@ extern "C" kivi_status kivi_decode_attn_noalloc(kivi_cache *c, const void *q, in
     kivi_status st = kivi::decode_params_external_scratch(c, q, H_q, out, &p, &D, &HG, &dtype,
                                                           &pre_rope, &rt, &ragged, &rows);
     if (st != KIVI_OK) return st;
-    const size_t tick_bytes = ((size_t)p.seqs * sizeof(int) + 255) / 256 * 256;
+    // One ticket per sequence and one per partial row (merge blocks).
+    const size_t tick_count = (size_t)p.seqs + (size_t)rows;
+    const size_t tick_bytes = (tick_count * sizeof(int) + 255) / 256 * 256;
     const size_t part_bytes = (size_t)rows * HG * (D + 4) * sizeof(float);
     if (tick_bytes + part_bytes > kNoAllocScratchBytes) return KIVI_ERR_CAPACITY;
     void *base = nullptr;
@@ -77,7 +79,7 @@ extern "C" kivi_status kivi_decode_attn_noalloc(kivi_cache *c, const void *q, in
     p.tickets = (int *)base;
     p.partials = (float *)((unsigned char *)base + tick_bytes);
     // The array keeps the previous call's contents: the tickets must start at 0.
-    e = cudaMemsetAsync(p.tickets, 0, (size_t)p.seqs * sizeof(int), (cudaStream_t)stream);
+    e = cudaMemsetAsync(p.tickets, 0, tick_count * sizeof(int), (cudaStream_t)stream);
     if (e == cudaSuccess)
         e = kivi::launch_decode(D, HG, dtype, pre_rope, p, ragged ? &rt : nullptr, (cudaStream_t)stream);
     return kivi::cuda_status(e);

@@ -188,9 +188,9 @@ KIVI_API kivi_status kivi_append_decode(kivi_cache *c, const void *k_t, const vo
  *     whose kernels overlap on the GPU (any caches, any streams) race on the
  *     array: order them, e.g. on one stream.
  *   - Returns KIVI_ERR_CAPACITY, launching nothing, when the call's scratch
- *     (tickets for B*H_kv sequences plus (warps + B*H_kv) partial rows of
- *     (H_q/H_kv)*(D+4) fp32, warps being the decode's work streams, at most
- *     the SM count times 16) exceeds the array.
+ *     (rows = warps + B*H_kv partial rows of (H_q/H_kv)*(D+4) fp32, warps
+ *     being the decode's work streams, at most the SM count times 16, plus
+ *     B*H_kv + rows int tickets) exceeds the array.
  * Arguments, layouts and other errors as kivi_decode_attn.
  */
 KIVI_API kivi_status kivi_decode_attn_noalloc(kivi_cache *c, const void *q, int H_q, float *out,

@@ -132,6 +132,42 @@ def test_pre_rope_longest_supported_context():
     run_stream(w, seed=6, steps=1)
 
 
+# Sequences split over many warps.  A sequence whose work spans more than 16
+# warps has its partials merged in two levels (blocks of 8 partials folded by
+# the last warp of each block, then the blocks by the last block); at most 16
+# are merged in one pass.  The cases put every warp on one sequence (thousands
+# of partials), a few hundred partials on each of eight sequences, and 17 or
+# 18 per sequence (140 sequences over 148 SMs x 16 warps), just past the
+# one-pass limit, where a sequence's last block can hold a single partial.
+SPLIT_CASES = [
+    ("llama2_7b_layer", dict(B=1, H_q=1, H_kv=1, T=60000), 2),
+    ("mistral_gqa", dict(B=1, H_q=32, H_kv=8, T=40000), 2),
+    ("llama2_7b_layer", dict(B=35, H_q=4, H_kv=4, T=1500), 2),
+    ("long_context", dict(B=1, H_q=8, H_kv=2, T=30000), 2),
+]
+
+
+@pytest.mark.parametrize("name,kw,steps", SPLIT_CASES,
+                         ids=["one-sequence", "gqa-8-sequences", "140-sequences", "pre-rope"])
+def test_sequences_split_over_many_warps(name, kw, steps):
+    w = small(name, steps=steps, **kw)
+    run_stream(w, seed=9, steps=steps)
+
+
+def test_two_level_merge_is_deterministic():
+    """The merge reads partials in slot order whichever warp finishes last, so
+    repeated decodes of a long sequence agree bit for bit."""
+    w = small("llama2_7b_layer", B=1, H_q=2, H_kv=2, T=50000, steps=0)
+    K, V = synth.prefill_inputs(w, 10, device=DEV)
+    c = KiviCache(w.B, w.H_kv, w.D, w.G, w.R, w.torch_dtype, w.T)
+    c.prefill(K, V)
+    q = synth.step_inputs(w, 0, 10, device=DEV)[2]
+    a = c.decode(q)
+    for _ in range(5):
+        assert torch.equal(c.decode(q), a)
+    assert c.device_status() == 0
+
+
 def test_head_dim_64_bf16_and_128_fp16():
     run_stream(small("tiny", dtype="bf16", T=400, B=2, steps=10), seed=5, steps=10)
     run_stream(small("llama2_7b_layer", dtype="fp16", T=400, B=1, H_q=2, H_kv=2, steps=10),

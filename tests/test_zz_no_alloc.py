@@ -45,6 +45,9 @@ def _call(fn, c, w, q):
 @pytest.mark.parametrize("name,kw,steps", [
     ("mistral_gqa", dict(B=4, H_q=16, H_kv=4, T=3000), 3),
     ("tiny", dict(B=3, H_q=2, H_kv=2, T=700), 130),
+    # two sequences over every warp: partials merged in two levels, with the
+    # merge blocks' tickets in the shared array too
+    ("llama2_7b_layer", dict(B=1, H_q=2, H_kv=2, T=20000), 1),
 ])
 def test_noalloc_matches_decode_attn_on_two_calls(name, kw, steps):
     torch.cuda.set_device(0)
