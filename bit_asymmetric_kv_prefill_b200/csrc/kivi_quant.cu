@@ -3,22 +3,29 @@
 // Keys are grouped per channel over 32 consecutive tokens and values per token
 // over 32 consecutive channels ("KIVI Quantization Secures Llama-2 Accuracy at
 // Two Bits", paragraphs 2-3; record kv-efficiency/kivi-2bit-llama2-13b-mha-4k,
-// "Quant method": kivi-2bit-per-channel-k-per-token-v).  Each CTA takes one
-// group tile (32 tokens x D channels of K and of V) at a time:
-//   1. the tile is staged into padded shared memory with cp.async, double
-//      buffered across the CTA's groups;
-//   2. statistics: per-channel key min/max with paired (bf16x2 / f16x2)
-//      min/max over 16 rows per thread, the two row halves merged by a warp
-//      shuffle; per-token value min/max over each 32-channel group;
+// "Quant method": kivi-2bit-per-channel-k-per-token-v).  One warp quantizes
+// one key tile or one value tile (32 tokens x D channels) at a time, holding
+// it in registers, and writes its half of the 24*D-byte group block; warps
+// never wait for each other:
+//   1. the tile is staged into the warp's shared buffer with cp.async (the
+//      next tile's copy overlaps the current tile's parameters and codes) and
+//      read row-wide into registers (keys: each lane takes D/32 channels of
+//      every token; values: each lane takes the CPL channels of 16 tokens
+//      that it owns in the block's code layout);
+//   2. statistics with paired (bf16x2 / f16x2) min/max: per key channel
+//      within the lane, per value token within the lane and then across the
+//      lanes of its 32-channel group by shuffles;
 //   3. each group's fp16 scale/zero and its three code thresholds.  The code
 //      clamp(rint(fl(x - z) / s), 0, 3) equals the number of thresholds x has
 //      reached, x_k being the smallest input value whose fp32 difference to z
 //      passes the k-th exact fp32 bound (see code_params); x_k is found by a
-//      bounded search around z + E_k that evaluates the definition itself;
+//      search from z + E_k that evaluates the definition itself;
 //   4. codes: two channels at a time, three paired `x >= x_k` compares give
-//      lane masks, two logic ops turn them into the pair's two 2-bit codes and
-//      one multiply-add shifts them into the word;
-//   5. the finished 24*D-byte group block leaves with coalesced 16-byte stores.
+//      lane masks, two logic ops turn them into the pair's two 2-bit codes at
+//      their word position; key words are assembled across the lanes that
+//      share them by shuffles;
+//   5. value code words leave as coalesced 16-byte stores, key words as
+//      4-byte stores that fill whole 16-byte chunks per warp store.
 // The residual rows of a prefill and the appended token of a flush are copied
 // by the same launch.
 #include <cstring>
@@ -107,10 +114,12 @@ __device__ __forceinline__ bool passes(uint16_t x, float e, float z)
 
 // Smallest input value x (as bits) with fl32(x - z) > e; +inf when none.
 // fl32(x - z) is non-decreasing in x, so {x : passes} is an upper set.  The
-// start c = RD_dtype(RD_fp32(z + e)) satisfies c - z <= e, so it never
-// passes; stepping up reaches the least passing value, normally in one or two
-// steps.  Should that not happen within 4 steps, a binary search over the
-// value-ordered 16-bit patterns settles it.
+// start c = RD_dtype(RD_fp32(z + e)) satisfies c - z <= e (rounding to
+// nearest is monotone and e is an fp32 value), so it never passes.  Its
+// successor x1 lies above z + e, so it passes whenever x1 - z is exact in
+// fp32, i.e. unless x1 and z are many binades apart; otherwise stepping on,
+// and after three more steps a binary search over the value-ordered 16-bit
+// patterns, settles it.
 template <int DT>
 __device__ __noinline__ uint16_t min_passing_slow(uint16_t x, float e, float z);
 
@@ -118,20 +127,22 @@ template <int DT>
 __device__ __forceinline__ uint16_t min_passing(float e, float z)
 {
     if (!(e < __int_as_float(0x7f800000))) return In<DT>::kInf;
-    // The first two steps, evaluated side by side; rarely more are needed.
-    const uint16_t x0 = In<DT>::from_float_rd(__fadd_rd(z, e));
-    const uint16_t x1 = next_up<DT>(x0), x2 = next_up<DT>(x1);
-    const bool p1 = passes<DT>(x1, e, z), p2 = passes<DT>(x2, e, z);
-    if (p1 | p2) return p1 ? x1 : x2;
-    return min_passing_slow<DT>(x2, e, z);
+    const uint16_t c = In<DT>::from_float_rd(__fadd_rd(z, e));
+    // The successor of c in value order (c is finite: a rounding down of a
+    // finite sum never gives +inf).
+    const uint16_t x1 = (c & 0x7fffu) == 0 ? (uint16_t)0x0001u
+                        : (c & 0x8000u)    ? (uint16_t)(c - 1)
+                                           : (uint16_t)(c + 1);
+    if (passes<DT>(x1, e, z)) return x1;
+    return min_passing_slow<DT>(x1, e, z);
 }
 
-// Continuation from x (not passing): two more steps, then a bisection.
+// Continuation from x (not passing): three more steps, then a bisection.
 template <int DT>
 __device__ __noinline__ uint16_t min_passing_slow(uint16_t x, float e, float z)
 {
 #pragma unroll 1
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 3; ++i) {
         x = next_up<DT>(x);
         if (passes<DT>(x, e, z)) return x;
     }
@@ -162,44 +173,6 @@ __device__ __forceinline__ uint32_t code_pair_bits(uint32_t x, uint32_t t1, uint
     asm("lop3.b32 %0, %1, %2, %3, 0x78;" : "=r"(r) : "r"(a), "r"(m2), "r"(0x00030003u));  // a^(m2&M)
     return r;
 }
-
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
-{
-    uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-constexpr int kQuantThreads = 256;
-#ifndef KIVI_QUANT_CTAS
-#define KIVI_QUANT_CTAS 4   // resident CTAs per SM (persistent grid; measured best)
-#endif
-
-// The CTA works as two independent halves: threads [0, D) take the key tile,
-// the rest the value tile, each with its own named barrier (ids 1 and 2), so
-// that neither waits for the other; the halves share only the SM.
-template <int D>
-__device__ __forceinline__ void half_sync(int tid)
-{
-    if (tid < D)
-        asm volatile("bar.sync 1, %0;" ::"n"(D) : "memory");
-    else
-        asm volatile("bar.sync 2, %0;" ::"n"(kQuantThreads - D) : "memory");
-}
-
-template <int D>
-struct QuantSmem {
-    static constexpr int RS = D + 8;                      // padded row, elements
-    static constexpr int TILE = 32 * RS;                  // one K or V tile
-    static constexpr int TILES_BYTES = 2 * 2 * TILE * 2;  // 2 buffers x (K, V)
-    static constexpr int THRK = TILES_BYTES;              // uint16 [3][D]
-    static constexpr int TS = 4 * (D / 32) + 4;           // padded token row of thrV
-    static constexpr int THRV = THRK + 3 * D * 2;         // uint16 [32][TS]: [D/32][4] + pad
-    static constexpr int OUTB = (THRV + 32 * TS * 2 + 15) / 16 * 16;
-    static constexpr int BYTES = OUTB + 24 * D;
-};
 
 // Work item of a quantizer launch: group g of sequence s (destination group
 // g_dst0 + g), or (copy) the residual copy of sequence s's source rows
@@ -252,261 +225,364 @@ __device__ __forceinline__ QItem locate(const QuantParams &p, const QuantSegs *s
     return q;
 }
 
-template <int D, int DT>
-__device__ void quantize_tile(const QuantParams &p, long long s, int g, long long g_dst0,
-                              const uint16_t *tk, const uint16_t *tv, uint16_t *thrK, uint16_t *thrV,
-                              uint8_t *outb)
+// ---- one warp per key tile or value tile ------------------------------------
+// Work unit 2*item is the key tile of group item, 2*item + 1 its value tile;
+// a warp takes units gw, gw + W, ... (W warps in the grid, even), so it
+// always works on one kind of tile.  A warp holds its tile in registers and
+// writes its own part of the group block; warps never wait for each other.
+
+// Two codes of a channel pair x against packed thresholds t1..t3, placed at
+// the word bits K1 (0x00010001 << 2i) and K3 (0x00030003 << 2i) of pair i.
+// Masks m_k are 0xffff per half where x >= t_k; as m1 >= m2 >= m3, bit 1 of
+// a code is m2 and bit 0 is m1 ^ m2 ^ m3.
+template <int DT>
+__device__ __forceinline__ uint32_t code_pair_at(uint32_t x, uint32_t t1, uint32_t t2, uint32_t t3, uint32_t K1,
+                                                 uint32_t K3)
+{
+    const uint32_t m1 = In<DT>::ge_mask(x, t1), m2 = In<DT>::ge_mask(x, t2), m3 = In<DT>::ge_mask(x, t3);
+    uint32_t a, r;
+    asm("lop3.b32 %0, %1, %2, %3, 0x28;" : "=r"(a) : "r"(m1), "r"(m3), "r"(K1));  // (m1^m3)&K1
+    asm("lop3.b32 %0, %1, %2, %3, 0x78;" : "=r"(r) : "r"(a), "r"(m2), "r"(K3));   // a^(m2&K3)
+    return r;
+}
+
+// Packed (a.lo, b.lo) and (a.hi, b.hi) of two 16-bit pairs.
+__device__ __forceinline__ uint32_t lo_halves(uint32_t a, uint32_t b) { return __byte_perm(a, b, 0x5410); }
+__device__ __forceinline__ uint32_t hi_halves(uint32_t a, uint32_t b) { return __byte_perm(a, b, 0x7632); }
+
+// Key tile: 32 tokens x D channels, one group per channel, staged in shared
+// memory.  Lane l holds the CK = D/32 channels [CK*l, CK*l + CK) of all 32
+// tokens (a whole row per warp load), so each channel's min/max,
+// scale, zero and thresholds are the lane's own.  The lane's channel pairs
+// are pairs i0, i0 + 1 of one 16-channel code word (a word of slice cs, local
+// channels 16k..16k+15); the 4 (D = 128) or 8 (D = 64) lanes of a word OR
+// their codes together in a transposing shuffle, which leaves each lane one
+// complete word per chunk of 4 or 8 tokens.
+template <int D, int DT, typename F>
+__device__ __forceinline__ void key_tile(const uint16_t *tile, uint8_t *blk, int lane, F &&after_stats)
 {
     using L = Layout<D>;
     using H = In<DT>;
-    constexpr int RS = QuantSmem<D>::RS;
-    constexpr int NJ = L::NJ, CPL = L::CPL, TPW = L::TPW, KW = L::KW;
-    const int tid = threadIdx.x;
+    constexpr int CK = D / 32, NP = CK / 2;
+    constexpr int NL = D == 128 ? 2 : 3;         // lanes per word = 2^NL
+    constexpr int CH = 1 << NL;                  // tokens per chunk
+    const int c0 = CK * lane;
 
-    if (tid < D) {
-        // Keys, per channel: thread (pair cp, row set hh) takes 16 rows of a
-        // channel pair, rows 8b + 4hh + {0..3} (the two sets 4 rows apart sit
-        // in disjoint banks); they meet through a shuffle with lane ^ 1.
-        const int cp = tid >> 1, hh = tid & 1;
-        const uint16_t *col = tk + hh * 4 * RS + 2 * cp;
-        auto row = [&](int i) { return (const uint32_t *)(col + (((i >> 2) << 3) + (i & 3)) * RS); };
-        uint32_t mn = *row(0), mx = mn;
-        uint32_t mn1 = *row(1), mx1 = mn1;
+    uint32_t x[32][NP];
 #pragma unroll
-        for (int r = 2; r < 16; r += 2) {
-            const uint32_t v0 = *row(r);
-            const uint32_t v1 = *row(r + 1);
-            mn = H::vmin(mn, v0);
-            mx = H::vmax(mx, v0);
-            mn1 = H::vmin(mn1, v1);
-            mx1 = H::vmax(mx1, v1);
-        }
-        mn = H::vmin(mn, mn1);
-        mx = H::vmax(mx, mx1);
-        mn = H::vmin(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
-        mx = H::vmax(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        const int ch = 2 * cp + hh;
-        const uint16_t mnb = (uint16_t)(hh ? mn >> 16 : mn), mxb = (uint16_t)(hh ? mx >> 16 : mx);
-        const CodeParams c = code_params(H::f(mnb), H::f(mxb));
-        thrK[ch] = min_passing<DT>(c.e1, c.z);
-        thrK[D + ch] = min_passing<DT>(c.e2, c.z);
-        thrK[2 * D + ch] = min_passing<DT>(c.e3, c.z);
-        const int off = L::KM + km_offset<D>(k_perm_index<D>(ch));
-        *(uint16_t *)(outb + off) = c.s_bits;
-        *(uint16_t *)(outb + off + D / 16) = c.z_bits;
-    } else {
-        // Values, per token: one (token, 32-channel group) per thread.
-        for (int qd = tid - D; qd < 32 * NJ; qd += kQuantThreads - D) {
-            const int t = qd / NJ, j = qd % NJ;
-            const uint4 *row = (const uint4 *)(tv + t * RS + j * 32);
-            uint4 a = row[0];
-            uint32_t mn = H::vmin(a.x, a.y), mx = H::vmax(a.x, a.y);
-            mn = H::vmin(mn, H::vmin(a.z, a.w));
-            mx = H::vmax(mx, H::vmax(a.z, a.w));
-#pragma unroll
-            for (int q = 1; q < 4; ++q) {
-                a = row[q];
-                mn = H::vmin(mn, H::vmin(H::vmin(a.x, a.y), H::vmin(a.z, a.w)));
-                mx = H::vmax(mx, H::vmax(H::vmax(a.x, a.y), H::vmax(a.z, a.w)));
-            }
-            mn = H::vmin(mn, (mn >> 16) | (mn << 16));
-            mx = H::vmax(mx, (mx >> 16) | (mx << 16));
-            const CodeParams c = code_params(H::f((uint16_t)mn), H::f((uint16_t)mx));
-            uint16_t *tr = thrV + t * QuantSmem<D>::TS + j * 4;
-            tr[0] = min_passing<DT>(c.e1, c.z);
-            tr[1] = min_passing<DT>(c.e2, c.z);
-            tr[2] = min_passing<DT>(c.e3, c.z);
-            const int off = L::VM + t * (D / 8) + j * 2;
-            *(uint16_t *)(outb + off) = c.s_bits;
-            *(uint16_t *)(outb + off + D / 16) = c.z_bits;
+    for (int t = 0; t < 32; ++t) {
+        if constexpr (NP == 2) {
+            const uint2 v = *(const uint2 *)(tile + t * D + c0);
+            x[t][0] = v.x;
+            x[t][1] = v.y;
+        } else {
+            x[t][0] = *(const uint32_t *)(tile + t * D + c0);
         }
     }
-    half_sync<D>(tid);
 
-    if (tid < D) {
-        // Key code words: thread -> (lane, token pair, word slot k); tokens tok
-        // and tok+2 of the lane share the word's 16 channels and thresholds.
-        const int lane = tid / (2 * KW), rem = tid % (2 * KW);
-        const int tokp = rem / KW, k = rem % KW;
-        const int cs = lane & 3, tq = lane >> 2;
-        // The word's 16 channels come in runs of RUN contiguous channels
-        // (one run when D >= 128, one per RoPE half when D == 64).
-        constexpr int RUN = L::HALF < 16 ? L::HALF : 16;
-        uint32_t t1[8], t2[8], t3[8];
-        int base[16 / RUN];
+    // Per channel pair: min/max over the 32 tokens, then each channel's
+    // parameters and thresholds (packed per pair: low half channel c, high
+    // half channel c + 1).
+    uint32_t T1[NP], T2[NP], T3[NP], mnp[NP], mxp[NP];
 #pragma unroll
-        for (int r = 0; r < 16 / RUN; ++r) {
-            base[r] = k_channel<D>(cs, 16 * k + r * RUN);
+    for (int pp = 0; pp < NP; ++pp) {
+        uint32_t mn[4], mx[4];
 #pragma unroll
-            for (int v = 0; v < RUN / 8; ++v) {
-                const uint4 a = *(const uint4 *)(thrK + base[r] + 8 * v);
-                const uint4 b = *(const uint4 *)(thrK + D + base[r] + 8 * v);
-                const uint4 c = *(const uint4 *)(thrK + 2 * D + base[r] + 8 * v);
-                const int i0 = r * (RUN / 2) + 4 * v;
-                t1[i0] = a.x; t1[i0 + 1] = a.y; t1[i0 + 2] = a.z; t1[i0 + 3] = a.w;
-                t2[i0] = b.x; t2[i0 + 1] = b.y; t2[i0 + 2] = b.z; t2[i0 + 3] = b.w;
-                t3[i0] = c.x; t3[i0 + 1] = c.y; t3[i0 + 2] = c.z; t3[i0 + 3] = c.w;
-            }
+        for (int a = 0; a < 4; ++a) mn[a] = mx[a] = x[a][pp];
+#pragma unroll
+        for (int t = 4; t < 32; ++t) {
+            mn[t & 3] = H::vmin(mn[t & 3], x[t][pp]);
+            mx[t & 3] = H::vmax(mx[t & 3], x[t][pp]);
         }
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int tok = tokp + 2 * h;
-            const uint16_t *row = tk + (4 * tq + tok) * RS;
-            uint32_t x[8];
-#pragma unroll
-            for (int r = 0; r < 16 / RUN; ++r)
-#pragma unroll
-                for (int v = 0; v < RUN / 8; ++v) {
-                    const uint4 a = *(const uint4 *)(row + base[r] + 8 * v);
-                    const int i0 = r * (RUN / 2) + 4 * v;
-                    x[i0] = a.x; x[i0 + 1] = a.y; x[i0 + 2] = a.z; x[i0 + 3] = a.w;
-                }
-            uint32_t word = 0;
-#pragma unroll
-            for (int i = 7; i >= 0; --i) word = word * 4u + code_pair_bits<DT>(x[i], t1[i], t2[i], t3[i]);
-            *(uint32_t *)(outb + L::KC + code_word_offset(lane, tok * KW + k)) = word;
-        }
-    } else {
-        // Value code words: thread -> (lane = 16*th + co, word u).
-        for (int vp = tid - D; vp < 2 * D; vp += kQuantThreads - D) {
-            const int lane = vp / L::WPL, u = vp % L::WPL;
-            const int co = lane & 15, th = lane >> 4;
-            const int j = co * CPL / 32;
-            // TPW tokens x CPL channels: per token one threshold triple (one
-            // 8-byte load) and CPL/2 channel pairs (CPL/8 16-byte loads).
-            uint32_t x[8], b1[TPW], b2[TPW], b3[TPW];
-#pragma unroll
-            for (int tt = 0; tt < TPW; ++tt) {
-                const int t = 16 * th + u * TPW + tt;
-                const uint2 tr = *(const uint2 *)(thrV + t * QuantSmem<D>::TS + j * 4);
-                b1[tt] = __byte_perm(tr.x, 0, 0x1010);
-                b2[tt] = __byte_perm(tr.x, 0, 0x3232);
-                b3[tt] = __byte_perm(tr.y, 0, 0x1010);
-                const uint16_t *row = tv + t * RS + co * CPL;
-                if constexpr (CPL >= 8) {
-#pragma unroll
-                    for (int v = 0; v < CPL / 8; ++v) {
-                        const uint4 a = *(const uint4 *)(row + 8 * v);
-                        const int i0 = tt * (CPL / 2) + 4 * v;
-                        x[i0] = a.x; x[i0 + 1] = a.y; x[i0 + 2] = a.z; x[i0 + 3] = a.w;
-                    }
-                } else {
-                    const uint2 a = *(const uint2 *)row;
-                    x[tt * 2] = a.x;
-                    x[tt * 2 + 1] = a.y;
-                }
-            }
-            uint32_t word = 0;
-#pragma unroll
-            for (int i = 7; i >= 0; --i) {
-                const int tt = i / (CPL / 2);
-                word = word * 4u + code_pair_bits<DT>(x[i], b1[tt], b2[tt], b3[tt]);
-            }
-            *(uint32_t *)(outb + L::VC + code_word_offset(lane, u)) = word;
-        }
+        mnp[pp] = H::vmin(H::vmin(mn[0], mn[1]), H::vmin(mn[2], mn[3]));
+        mxp[pp] = H::vmax(H::vmax(mx[0], mx[1]), H::vmax(mx[2], mx[3]));
     }
-    half_sync<D>(tid);
-
-    // Each half stores its own 12*D bytes: [Kc, Km) and [Vc, Vm).
-    uint4 *dst = (uint4 *)(p.packed + ((s * p.ngcap) + g_dst0 + g) * (long long)L::GB);
-    {
-        const int h = tid < D ? 0 : 1, ht = tid < D ? tid : tid - D;
-        const int nthr = tid < D ? D : kQuantThreads - D;
-        const uint4 *src = (const uint4 *)(outb + h * 12 * D);
-        uint4 *d = dst + h * (12 * D / 16);
-        for (int c = ht; c < 12 * D / 16; c += nthr) d[c] = src[c];
+    after_stats();
+    // One channel per iteration (a loop, to keep the code small): its 16-bit
+    // min/max shift out of mn64/mx64 and its results shift into t*s, ss, zs.
+    uint64_t mn64 = mnp[0], mx64 = mxp[0];
+    if constexpr (NP == 2) {
+        mn64 |= (uint64_t)mnp[1] << 32;
+        mx64 |= (uint64_t)mxp[1] << 32;
+    }
+    uint64_t t1s = 0, t2s = 0, t3s = 0, ss = 0, zs = 0;
+#pragma unroll 1
+    for (int ch = 0; ch < CK; ++ch) {
+        const CodeParams c = code_params(H::f((uint16_t)mn64), H::f((uint16_t)mx64));
+        mn64 >>= 16;
+        mx64 >>= 16;
+        const int sh = 16 * ch;
+        t1s |= (uint64_t)min_passing<DT>(c.e1, c.z) << sh;
+        t2s |= (uint64_t)min_passing<DT>(c.e2, c.z) << sh;
+        t3s |= (uint64_t)min_passing<DT>(c.e3, c.z) << sh;
+        ss |= (uint64_t)c.s_bits << sh;
+        zs |= (uint64_t)c.z_bits << sh;
+    }
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+        T1[pp] = (uint32_t)(t1s >> (32 * pp));
+        T2[pp] = (uint32_t)(t2s >> (32 * pp));
+        T3[pp] = (uint32_t)(t3s >> (32 * pp));
+        // Channels c, c + 1 have consecutive permuted indices (even first).
+        const int off = L::KM + km_offset<D>(k_perm_index<D>(c0 + 2 * pp));
+        *(uint32_t *)(blk + off) = (uint32_t)(ss >> (32 * pp));
+        *(uint32_t *)(blk + off + D / 16) = (uint32_t)(zs >> (32 * pp));
     }
 
-    if (p.newK != nullptr && g == 0) {
-        // The flush has read residual slot 0 into shared memory (each half's
-        // tile was complete before that half's first barrier): the new token
-        // may land, each half writing its own row.
-        const int which = tid < D ? 0 : 1, ht = tid < D ? tid : tid - D;
-        for (int q = ht; q < D / 8; q += (tid < D ? D : kQuantThreads - D)) {
-            const uint16_t *src = (which ? p.newV : p.newK) + s * D + q * 8;
-            uint16_t *d = (which ? p.resV : p.resK) + s * (long long)p.R * D + q * 8;
-            *(uint4 *)d = *(const uint4 *)src;
+    // Word position of the lane's pairs and of its words after the exchange.
+    const int P0 = k_perm_index<D>(c0);
+    const int cs = P0 / (D / 4), L0 = P0 % (D / 4);
+    const int k = L0 / 16, i0 = (L0 % 16) / 2;
+    uint32_t K1[NP], K3[NP];
+#pragma unroll
+    for (int pp = 0; pp < NP; ++pp) {
+        K1[pp] = 0x00010001u << (2 * (i0 + pp));
+        K3[pp] = 0x00030003u << (2 * (i0 + pp));
+    }
+    // Lane bit of exchange level r: 0, 1 and (D = 64) 4; token offset kept.
+    constexpr int LB[3] = {0, 1, 4};
+    int jt = 0;
+#pragma unroll
+    for (int r = 0; r < NL; ++r) jt |= ((lane >> LB[r]) & 1) << r;
+    const int off0 = L::KC + code_word_offset(4 * (jt / 4) + cs, (jt % 4) * L::KW + k);
+
+#pragma unroll
+    for (int m = 0; m < 32 / CH; ++m) {
+        uint32_t w[CH];
+#pragma unroll
+        for (int q = 0; q < CH; ++q) {
+            const int t = m * CH + q;
+            uint32_t acc = 0;
+#pragma unroll
+            for (int pp = 0; pp < NP; ++pp) acc |= code_pair_at<DT>(x[t][pp], T1[pp], T2[pp], T3[pp], K1[pp], K3[pp]);
+            w[q] = acc;
         }
+#pragma unroll
+        for (int r = 0; r < NL; ++r) {
+            const bool b = (lane >> LB[r]) & 1;
+#pragma unroll
+            for (int e = 0; e < (CH >> (r + 1)); ++e) {
+                const uint32_t lo = w[2 * e], hi = w[2 * e + 1];
+                const uint32_t send = b ? lo : hi, keep = b ? hi : lo;
+                w[e] = keep | __shfl_xor_sync(0xffffffffu, send, 1 << LB[r]);
+            }
+        }
+        // w[0]: the word of token m*CH + jt (layout lane 4*(t/4) + cs, word
+        // (t%4)*KW + k); consecutive chunks are CH*16 bytes apart.
+        *(uint32_t *)(blk + off0 + m * CH * 16) = w[0];
     }
 }
 
-template <int D, int DT, bool SEG>
-__device__ __forceinline__ void quant_body(const QuantParams &p, const QuantSegs *sg)
+// Value tile: 32 tokens x D channels, one group per (token, 32 channels).
+// Lane l = 16*th + co holds exactly what it owns in the block's value codes:
+// channels [co*CPL, (co+1)*CPL) of tokens 16th..16th+15.  A token's group
+// spans LG = 32/CPL lanes; they reduce its (min, -max) in a transposing
+// shuffle that leaves each lane 16/LG of the tokens, whose parameters it
+// computes and publishes (thresholds replicated in both halves) in the warp's
+// shared array `thr` [32 tokens][NJ].
+template <int D, int DT, typename F>
+__device__ __forceinline__ void value_tile(const uint16_t *tile, uint8_t *blk, int lane, uint4 *thr,
+                                           F &&after_stats)
 {
-    using S = QuantSmem<D>;
-    extern __shared__ __align__(16) unsigned char smem[];
-    uint16_t *tiles = (uint16_t *)smem;
-    uint16_t *thrK = (uint16_t *)(smem + S::THRK);
-    uint16_t *thrV = (uint16_t *)(smem + S::THRV);
-    uint8_t *outb = smem + S::OUTB;
+    using L = Layout<D>;
+    using H = In<DT>;
+    constexpr int CPL = L::CPL, NPV = CPL / 2, TPW = L::TPW, NJ = L::NJ, WPL = L::WPL;
+    constexpr int LG = kG / CPL;              // lanes per value group
+    constexpr int NLV = LG == 4 ? 2 : 3;      // log2(LG)
+    constexpr int TL = 16 / LG;               // tokens per lane after the exchange
+    const int co = lane & 15, th = lane >> 4;
+    const int j = co * CPL / kG, jl = lane & (LG - 1);
 
+    uint32_t x[16][NPV];
+    const uint16_t *base = tile + (16 * th) * D + co * CPL;
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt) {
+        if constexpr (NPV == 4) {
+            const uint4 v = *(const uint4 *)(base + tt * D);
+            x[tt][0] = v.x;
+            x[tt][1] = v.y;
+            x[tt][2] = v.z;
+            x[tt][3] = v.w;
+        } else {
+            const uint2 v = *(const uint2 *)(base + tt * D);
+            x[tt][0] = v.x;
+            x[tt][1] = v.y;
+        }
+    }
+
+    // (min, -max) of each token over the lane's channels, packed.
+    uint32_t M[16];
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt) {
+        uint32_t mn = x[tt][0], mx = x[tt][0];
+#pragma unroll
+        for (int pp = 1; pp < NPV; ++pp) {
+            mn = H::vmin(mn, x[tt][pp]);
+            mx = H::vmax(mx, x[tt][pp]);
+        }
+        const uint32_t nmx = mx ^ 0x80008000u;
+        M[tt] = H::vmin(lo_halves(mn, nmx), hi_halves(mn, nmx));
+    }
+    after_stats();
+    // Over the LG lanes of the group: level r keeps the tokens whose bit r is
+    // the lane's bit r.  M[m] then holds token m*LG + jl.
+#pragma unroll
+    for (int r = 0; r < NLV; ++r) {
+        const bool b = (lane >> r) & 1;
+#pragma unroll
+        for (int e = 0; e < (16 >> (r + 1)); ++e) {
+            const uint32_t lo = M[2 * e], hi = M[2 * e + 1];
+            const uint32_t send = b ? lo : hi, keep = b ? hi : lo;
+            M[e] = H::vmin(keep, __shfl_xor_sync(0xffffffffu, send, 1 << r));
+        }
+    }
+    __syncwarp();   // the previous tile's thresholds have been read
+    // One token per iteration (a loop, to keep the code small): M rotates.
+#pragma unroll 1
+    for (int m = 0; m < TL; ++m) {
+        const uint32_t cur = M[0];
+#pragma unroll
+        for (int k = 0; k + 1 < TL; ++k) M[k] = M[k + 1];
+        const int t = 16 * th + m * LG + jl;
+        const float mnf = H::f((uint16_t)cur);
+        const float mxf = -H::f((uint16_t)(cur >> 16));
+        const CodeParams c = code_params(mnf, mxf);
+        const uint32_t t1 = min_passing<DT>(c.e1, c.z), t2 = min_passing<DT>(c.e2, c.z),
+                       t3 = min_passing<DT>(c.e3, c.z);
+        thr[t * NJ + j] = make_uint4(t1 * 0x10001u, t2 * 0x10001u, t3 * 0x10001u, 0u);
+        const int off = L::VM + t * (D / 8) + j * 2;
+        *(uint16_t *)(blk + off) = c.s_bits;
+        *(uint16_t *)(blk + off + D / 16) = c.z_bits;
+    }
+    __syncwarp();
+
+    // Word u: tokens 16th + u*TPW + q, pair i = q*NPV + pp at bits 2i, 16+2i.
+    uint32_t wv[WPL];
+#pragma unroll
+    for (int u = 0; u < WPL; ++u) {
+        uint4 b[TPW];
+#pragma unroll
+        for (int q = 0; q < TPW; ++q) b[q] = thr[(16 * th + u * TPW + q) * NJ + j];
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+            const int q = i / NPV, pp = i % NPV;
+            word = word * 4u + code_pair_bits<DT>(x[u * TPW + q][pp], b[q].x, b[q].y, b[q].z);
+        }
+        wv[u] = word;
+    }
+#pragma unroll
+    for (int c = 0; c < WPL / 4; ++c)
+        *(uint4 *)(blk + L::VC + (c * 32 + lane) * 16) = make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+}
+
+constexpr int kQuantWarps = 8;   // warps per CTA
+
+// Shared memory per warp: the staged tile (32 rows of D), then the value
+// tile's thresholds [32 tokens][NJ].
+template <int D>
+struct QuantWarpSmem {
+    static constexpr int TILE = 32 * D * 2;
+    static constexpr int THR = 32 * Layout<D>::NJ * 16;
+    static constexpr int PER_WARP = TILE + THR;
+    static constexpr int BYTES = kQuantWarps * PER_WARP;
+};
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// A warp's units, one after another; the tile of the next unit is staged into
+// the warp's buffer (cp.async) as soon as the current tile's statistics have
+// consumed the buffer, so its load overlaps the parameters and codes.
+template <int D, int DT, bool SEG>
+__device__ __forceinline__ void quant_warps(const QuantParams &p, const QuantSegs *sg)
+{
+    using S = QuantWarpSmem<D>;
+    extern __shared__ __align__(16) unsigned char qsm[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint16_t *tile = (uint16_t *)(qsm + wid * S::PER_WARP);
+    uint4 *thr = (uint4 *)(qsm + wid * S::PER_WARP + S::TILE);
     long long n_items;
     if constexpr (SEG) n_items = sg->item0[sg->nseg];
     else n_items = p.seqs * (long long)p.n_g + (p.r_copy > 0 ? p.seqs : 0);
-    const int tid = threadIdx.x;
+    const long long n_units = 2 * n_items;
+    const long long nw = (long long)gridDim.x * kQuantWarps;
 
-    auto issue = [&](long long item, int buf) {
-        if (item >= n_items) return;
-        const QItem q = locate<SEG>(p, sg, item);
+    // Stage unit u's tile (nothing for a copy item).
+    auto stage = [&](const QItem &q, bool vhalf) {
         if (q.copy) return;
-        const long long s = q.s;
-        const int g = q.g;
-        const long long row0 = s * p.src_seq_rows + (long long)g * 32;
-        const uint16_t *k = p.srcK + row0 * D;
-        const uint16_t *v = p.srcV + row0 * D;
-        // The key half copies the key tile, the value half the value tile.
-        const bool kh = tid < D;
-        uint16_t *t = tiles + (buf * 2 + (kh ? 0 : 1)) * S::TILE;
-        const uint16_t *src = kh ? k : v;
-        const int ht = kh ? tid : tid - D, nthr = kh ? D : kQuantThreads - D;
-        for (int c = ht; c < 32 * (D / 8); c += nthr) {
-            const int row = c / (D / 8), col = (c % (D / 8)) * 8;
-            cp_async16(t + row * S::RS + col, src + row * D + col);
-        }
+        const uint4 *src =
+            (const uint4 *)((vhalf ? p.srcV : p.srcK) + (q.s * p.src_seq_rows + (long long)q.g * 32) * D);
+#pragma unroll
+        for (int c = 0; c < S::TILE / 16 / 32; ++c) cp_async16((uint4 *)tile + c * 32 + lane, src + c * 32 + lane);
     };
 
-    long long item = blockIdx.x;
-    int buf = 0;
-    issue(item, 0);
+    long long unit = (long long)blockIdx.x * kQuantWarps + wid;
+    const bool vhalf = unit & 1;   // nw is even: a warp keeps its kind of tile
+    if (unit >= n_units) return;
+    QItem q = locate<SEG>(p, sg, unit >> 1);
+    stage(q, vhalf);
     cp_async_commit();
-    for (; item < n_items; item += gridDim.x, buf ^= 1) {
-        issue(item + gridDim.x, buf ^ 1);
-        cp_async_commit();
-        cp_async_wait<1>();
-        half_sync<D>(tid);
-        const QItem q = locate<SEG>(p, sg, item);
-        if (!q.copy) {
-            quantize_tile<D, DT>(p, q.s, q.g, q.g_dst0, tiles + (buf * 2 + 0) * S::TILE,
-                                 tiles + (buf * 2 + 1) * S::TILE, thrK, thrV, outb);
+    for (;;) {
+        const long long next = unit + nw;
+        const bool has_next = next < n_units;
+        QItem qn = q;
+        if (has_next) qn = locate<SEG>(p, sg, next >> 1);
+        // After the current tile's statistics: stage the next tile.
+        auto after_stats = [&]() {
+            __syncwarp();
+            if (has_next) stage(qn, vhalf);
+            cp_async_commit();
+        };
+        if (q.copy) {
+            // Prefill residual: source rows [copy_row0, copy_row0 + r_copy) -> slots.
+            after_stats();
+            const uint4 *sr = (const uint4 *)((vhalf ? p.srcV : p.srcK) + (q.s * p.src_seq_rows + q.copy_row0) * D);
+            uint4 *dr = (uint4 *)((vhalf ? p.resV : p.resK) + q.s * (long long)p.R * D);
+            const int n16 = q.r_copy * (D / 8);
+            for (int c = lane; c < n16; c += 32) dr[c] = __ldcs(sr + c);
         } else {
-            // Prefill residual: rows [copy_row0, copy_row0 + r_copy) -> slots.
-            const long long s = q.s;
-            const long long n16 = (long long)q.r_copy * (D / 8);
-            const uint4 *sk = (const uint4 *)(p.srcK + (s * p.src_seq_rows + q.copy_row0) * D);
-            const uint4 *sv = (const uint4 *)(p.srcV + (s * p.src_seq_rows + q.copy_row0) * D);
-            uint4 *dk = (uint4 *)(p.resK + s * (long long)p.R * D);
-            uint4 *dv = (uint4 *)(p.resV + s * (long long)p.R * D);
-            const bool kh = tid < D;
-            const uint4 *sr = kh ? sk : sv;
-            uint4 *dr = kh ? dk : dv;
-            for (long long c = kh ? tid : tid - D; c < n16; c += kh ? D : kQuantThreads - D) dr[c] = sr[c];
+            cp_async_wait_all();
+            __syncwarp();
+            uint8_t *blk = p.packed + (q.s * p.ngcap + q.g_dst0 + q.g) * (long long)Layout<D>::GB;
+            if (!vhalf) key_tile<D, DT>(tile, blk, lane, after_stats);
+            else value_tile<D, DT>(tile, blk, lane, thr, after_stats);
+            if (p.newK != nullptr && q.g == 0) {
+                // A flush: the tile (residual slots 0..31) was read before
+                // its statistics, so the new token may replace slot 0 (the
+                // key warp its key row, the value warp its value row).
+                const uint4 *ns = (const uint4 *)((vhalf ? p.newV : p.newK) + q.s * D);
+                uint4 *nd = (uint4 *)((vhalf ? p.resV : p.resK) + q.s * (long long)p.R * D);
+                for (int c = lane; c < D / 8; c += 32) nd[c] = ns[c];
+            }
         }
-        half_sync<D>(tid);
+        if (!has_next) break;
+        unit = next;
+        q = qn;
     }
-    cp_async_wait<0>();
+    cp_async_wait_all();
 }
 
+#ifndef KIVI_QUANT_CTAS
+#define KIVI_QUANT_CTAS 2   // resident CTAs of 8 warps per SM (persistent grid)
+#endif
+
 template <int D, int DT>
-__global__ void __launch_bounds__(kQuantThreads, KIVI_QUANT_CTAS) quant_kernel(QuantParams p)
+__global__ void __launch_bounds__(kQuantWarps * 32, KIVI_QUANT_CTAS) quant_kernel(QuantParams p)
 {
-    quant_body<D, DT, false>(p, nullptr);
+    quant_warps<D, DT, false>(p, nullptr);
 }
 
 template <int D, int DT>
-__global__ void __launch_bounds__(kQuantThreads, KIVI_QUANT_CTAS)
+__global__ void __launch_bounds__(kQuantWarps * 32, KIVI_QUANT_CTAS)
     quant_kernel_seg(QuantParams p, const __grid_constant__ QuantSegs sg)
 {
-    quant_body<D, DT, true>(p, &sg);
+    quant_warps<D, DT, true>(p, &sg);
 }
 
 // Plain append: token rows [seqs][D] -> residual slot `slot` of each sequence.
@@ -552,24 +628,26 @@ int num_sms()
 template <int D, int DT>
 static cudaError_t launch_quant_t(const QuantParams &p, const QuantSegs *segs, cudaStream_t st)
 {
-    using S = QuantSmem<D>;
     const long long items = segs ? segs->item0[segs->nseg]
                                  : p.seqs * (long long)p.n_g + (p.r_copy > 0 ? p.seqs : 0);
     if (items == 0) return cudaSuccess;
+    // Two work units (key tile, value tile) per item, one warp each.
     long long grid = (long long)num_sms() * KIVI_QUANT_CTAS;
-    if (grid > items) grid = items;
+    const long long need = (2 * items + kQuantWarps - 1) / kQuantWarps;
+    if (grid > need) grid = need;
     QuantParams q = p;
     q.div_ng = make_magic((unsigned long long)(p.n_g > 0 ? p.n_g : 1));
+    using S = QuantWarpSmem<D>;
     if (segs) {
         static PerDeviceOnce once;
         const cudaError_t e = set_smem_once(once, quant_kernel_seg<D, DT>, S::BYTES);
         if (e != cudaSuccess) return e;
-        quant_kernel_seg<D, DT><<<(unsigned)grid, kQuantThreads, S::BYTES, st>>>(q, *segs);
+        quant_kernel_seg<D, DT><<<(unsigned)grid, kQuantWarps * 32, S::BYTES, st>>>(q, *segs);
     } else {
         static PerDeviceOnce once;
         const cudaError_t e = set_smem_once(once, quant_kernel<D, DT>, S::BYTES);
         if (e != cudaSuccess) return e;
-        quant_kernel<D, DT><<<(unsigned)grid, kQuantThreads, S::BYTES, st>>>(q);
+        quant_kernel<D, DT><<<(unsigned)grid, kQuantWarps * 32, S::BYTES, st>>>(q);
     }
     return cudaGetLastError();
 }
