@@ -226,10 +226,12 @@ __device__ __forceinline__ QItem locate(const QuantParams &p, const QuantSegs *s
 }
 
 // ---- one warp per key tile or value tile ------------------------------------
-// Work unit 2*item is the key tile of group item, 2*item + 1 its value tile;
-// a warp takes units gw, gw + W, ... (W warps in the grid, even), so it
-// always works on one kind of tile.  A warp holds its tile in registers and
-// writes its own part of the group block; warps never wait for each other.
+// Work unit 2*item is the key tile of group item, 2*item + 1 its value tile
+// (or, for a copy item, its key and value rows); a warp takes the units at
+// positions gw, gw + W, ... (W warps in the grid, even) counted from the last
+// unit down, so it always works on one kind of tile.  A warp holds its tile
+// in registers and writes its own part of the group block; warps never wait
+// for each other.
 
 // Two codes of a channel pair x against packed thresholds t1..t3, placed at
 // the word bits K1 (0x00010001 << 2i) and K3 (0x00030003 << 2i) of pair i.
@@ -513,6 +515,9 @@ __device__ __forceinline__ void quant_warps(const QuantParams &p, const QuantSeg
     const long long n_units = 2 * n_items;
     const long long nw = (long long)gridDim.x * kQuantWarps;
 
+    // Units run from the last down, so that the residual copies (the last
+    // items) start first and overlap the tiles.
+    auto item_of = [&](long long unit) { return (n_units - 1 - unit) >> 1; };
     // Stage unit u's tile (nothing for a copy item).
     auto stage = [&](const QItem &q, bool vhalf) {
         if (q.copy) return;
@@ -523,16 +528,18 @@ __device__ __forceinline__ void quant_warps(const QuantParams &p, const QuantSeg
     };
 
     long long unit = (long long)blockIdx.x * kQuantWarps + wid;
-    const bool vhalf = unit & 1;   // nw is even: a warp keeps its kind of tile
+    // Position unit runs work unit n_units - 1 - unit (value tile when odd);
+    // nw is even, so a warp keeps its kind of tile.
+    const bool vhalf = (n_units - 1 - unit) & 1;
     if (unit >= n_units) return;
-    QItem q = locate<SEG>(p, sg, unit >> 1);
+    QItem q = locate<SEG>(p, sg, item_of(unit));
     stage(q, vhalf);
     cp_async_commit();
     for (;;) {
         const long long next = unit + nw;
         const bool has_next = next < n_units;
         QItem qn = q;
-        if (has_next) qn = locate<SEG>(p, sg, next >> 1);
+        if (has_next) qn = locate<SEG>(p, sg, item_of(next));
         // After the current tile's statistics: stage the next tile.
         auto after_stats = [&]() {
             __syncwarp();
@@ -540,12 +547,23 @@ __device__ __forceinline__ void quant_warps(const QuantParams &p, const QuantSeg
             cp_async_commit();
         };
         if (q.copy) {
-            // Prefill residual: source rows [copy_row0, copy_row0 + r_copy) -> slots.
-            after_stats();
+            // Prefill residual: source rows [copy_row0, copy_row0 + r_copy)
+            // -> slots, 32 rows at a time through the warp's buffer (one
+            // round trip to memory per 32 rows), then the next tile is staged.
             const uint4 *sr = (const uint4 *)((vhalf ? p.srcV : p.srcK) + (q.s * p.src_seq_rows + q.copy_row0) * D);
             uint4 *dr = (uint4 *)((vhalf ? p.resV : p.resK) + q.s * (long long)p.R * D);
-            const int n16 = q.r_copy * (D / 8);
-            for (int c = lane; c < n16; c += 32) dr[c] = __ldcs(sr + c);
+            uint4 *buf = (uint4 *)tile;
+            for (int r0 = 0; r0 < q.r_copy; r0 += 32) {
+                const int n16 = (q.r_copy - r0 < 32 ? q.r_copy - r0 : 32) * (D / 8);
+                const int c0 = r0 * (D / 8);
+                for (int c = lane; c < n16; c += 32) cp_async16(buf + c, sr + c0 + c);
+                cp_async_commit();
+                cp_async_wait_all();
+                __syncwarp();
+                for (int c = lane; c < n16; c += 32) dr[c0 + c] = buf[c];
+                __syncwarp();
+            }
+            after_stats();
         } else {
             cp_async_wait_all();
             __syncwarp();
