@@ -122,9 +122,12 @@ struct DecodeShape {
     // that are multiples of 4 use them best: 12 warps leave 168 registers a
     // thread, 8 leave 255.  Pre-RoPE keys with four or more query heads per
     // kv head need more than 168 (measured 12.6% faster at 8 warps, 4 stages);
-    // without RoPE, 12 warps are faster despite a few spilled registers.
-    static constexpr int CAP = HG >= 4 ? (ROPE ? KIVI_DECODE_MAXW_GQA_ROPE : KIVI_DECODE_MAXW_GQA)
-                                       : KIVI_DECODE_MAXW;
+    // so do eight query heads per kv head (1.5 KB of spills at 12 warps;
+    // 364 -> 225 us at 8 warps on a 16 x 8-kv-head, 8K-token cache); four
+    // heads without RoPE fit 168 and run faster at 12 warps.
+    static constexpr int CAP = HG >= 8   ? KIVI_DECODE_MAXW_GQA_ROPE
+                               : HG >= 4 ? (ROPE ? KIVI_DECODE_MAXW_GQA_ROPE : KIVI_DECODE_MAXW_GQA)
+                                         : KIVI_DECODE_MAXW;
     static constexpr int NW = MAXW > CAP ? CAP : MAXW;   // warps per SM
     // Warps per CTA: a CTA of CW warps, NW / CW of them per SM.  A smaller CTA
     // leaves the SM as soon as its own warps are done, so the next launch (a
