@@ -207,3 +207,40 @@ def test_fake_quant_binding_rejects_host_tensors():
         kivi.fake_quant(torch.zeros(4, 64, 128, dtype=torch.bfloat16), kivi.AXIS_PER_CHANNEL)
     with pytest.raises(ValueError):
         kivi.fake_quant(torch.zeros(128, dtype=torch.bfloat16), kivi.AXIS_PER_TOKEN)
+
+
+@pytest.mark.parametrize("seqs,n_groups,r,warps", [
+    (1, 1871, 34, 2368),     # every warp on one sequence
+    (8, 1250, 2, 1776),      # a few hundred partials per sequence
+    (140, 44, 94, 2368),     # 17 or 18 partials: just past one pass, a last block of one
+    (256, 124, 128, 2368),   # Llama-2-7B layer: one pass everywhere
+    (3, 0, 7, 2),
+    (37, 900, 5, 1184),
+])
+def test_merge_rows_and_tickets_stay_in_their_arrays(seqs, n_groups, r, warps):
+    """Scratch bounds of the decode merge: sequence s's partial of slot k sits
+    at row first(s) + s + k, and when the sequence spans more than 16 warps
+    its merge blocks of 8 slots take tickets seqs + first(s) + s + kb.  Every
+    row lies below warps + seqs (the rows the library reserves), every ticket
+    below seqs + warps + seqs, and no row or ticket serves two sequences."""
+    F = 8
+    warps = min(warps, seqs * (n_groups * 4 + -(-r // 6) * 3))
+    rows, tickets = set(), set()
+    for s in range(seqs):
+        first, last, _, _ = kivi.decode_split(seqs, n_groups, r, 4, 3, warps, s, 0)
+        count = last - first + 1
+        if count == 1:
+            continue   # written directly, no partial
+        for k in range(count):
+            row = first + s + k
+            assert 0 <= row < warps + seqs
+            assert row not in rows
+            rows.add(row)
+        assert s not in tickets
+        tickets.add(s)
+        if count > 2 * F:
+            for kb in range(-(-count // F)):
+                t = seqs + first + s + kb
+                assert seqs <= t < seqs + warps + seqs
+                assert t not in tickets
+                tickets.add(t)
